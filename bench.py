@@ -1,0 +1,518 @@
+"""Benchmark of the ternary decode GEMV hot path on B200.
+
+Workload (one "step"): the 8B-class decode layer set at batch 1 in both packed layouts — GEMVs
+N x K = 4096 x 4096 (attention projection), 24576 x 4096 (fused gate/up), 4096 x 12288 (down),
+each in Q2_0_g128 and in base-3 (5 trits/byte) — i.e. six tern_gemv calls per step. Inputs are
+seeded synthetic codes (P(0)=0.4, P(+-1)=0.3), scales fp16(|N(0,1)|*0.02), activations fp16(N(0,1)).
+Metric: algorithmic bytes (packed codes + fp16 scales + x + y) per second, GB/s, whole job.
+
+L2 policy: the step rotates over enough copies of the weights that the footprint exceeds 3x the
+L2 size, so every step reads its weights from HBM. Device time comes from CUDA events on the
+launching stream around exactly --steps graph replays, with a barrier + synchronize on both sides
+and the max over ranks. Multi-GPU runs are independent replicas (weak scaling, no data-path
+collective). The e2e figure repeats the step through the public API with host-resident
+activations (pinned) copied in and results copied out inside the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--no-extras]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+LAYER_SET = [(4096, 4096), (24576, 4096), (4096, 12288)]  # (N, K) of the 8B-class decode layers
+GROUP = 128
+L2_BYTES_DEFAULT = 126 * 1024 * 1024
+METRIC = "ternary GEMV GB/s (weights/s) & % of 8 TB/s HBM; GEMM TFLOP/s vs fp16 peak"
+WORKLOAD = "8B-class decode layer set, batch 1, Q2_0_g128 + base-3: 4096x4096, 24576x4096, 4096x12288"
+
+
+def _env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=50)
+    p.add_argument("--impl", default="native", choices=["native", "reference"])
+    p.add_argument("--no-extras", action="store_true", help="skip the per-row measurements of the other kernels")
+    p.add_argument("--profile-step", action="store_true", help="few launches, for an ncu launch list")
+    return p.parse_args()
+
+
+# ------------------------------------------------------------------------------------- helpers
+def algorithmic_bytes(layout: int, n: int, k: int, batch: int) -> int:
+    """Bytes a GEMV must move: packed code rows + k/128 fp16 scales per row + x + y."""
+    import gemm_tern_gemv_b200 as T
+    return n * T.row_bytes(layout, k) + n * (k // GROUP) * 2 + batch * k * 2 + batch * n * 2
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def source_digest(name: str) -> str:
+    import hashlib
+    with open(os.path.join(ROOT, "gemm_tern_gemv_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(kernel_key: str):
+    """dram bytes per launch from the committed ncu summary, if taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[kernel_key]
+        if e.get("source_sha") == source_digest(e["source"]):
+            return e["dram_bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """Samples nvidia-smi SM clock / throttle reasons every 200 ms while active."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+# ----------------------------------------------------------------------------- the native arm
+def make_weights(torch, T, n, k, layout, seed, device):
+    """Seeded synthetic packed weights generated on the device and packed with tern_pack."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    u = torch.rand((n, k), generator=g, device=device)
+    t = torch.where(u < 0.3, -1.0, torch.where(u < 0.7, 0.0, 1.0))
+    s = (torch.randn((n, k // GROUP), generator=g, device=device).abs() * 0.02).to(torch.float16)
+    w = (t * s.float().repeat_interleave(GROUP, dim=1)).to(torch.float16)  # exact: s * t
+    del u, t
+    return T.pack(w, s, layout)
+
+
+def run_native(args, rank, world, local_rank):
+    import torch
+    import gemm_tern_gemv_b200 as T
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    T.lib()
+    peaks = load_peaks()
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", L2_BYTES_DEFAULT) or L2_BYTES_DEFAULT
+
+    layouts = [T.Q2_0_G128, T.T3_5PB_G128]
+    mats = [(layout, n, k) for layout in layouts for (n, k) in LAYER_SET]
+    set_bytes = sum(algorithmic_bytes(l, n, k, 1) for (l, n, k) in mats)
+    weight_bytes = sum(n * T.row_bytes(l, k) + n * (k // GROUP) * 2 for (l, n, k) in mats)
+    copies = max(2, math.ceil(3 * l2 / weight_bytes))
+
+    # weights: `copies` independent copies of every matrix (distinct memory, same distribution)
+    W = [[make_weights(torch, T, n, k, l, 1000 * c + 10 * i + rank, dev) for i, (l, n, k) in enumerate(mats)]
+         for c in range(copies)]
+    xs = [torch.randn((1, k), device=dev).to(torch.float16) for (_, _, k) in mats]
+    ys = [torch.empty((1, n), dtype=torch.float16, device=dev) for (_, n, _) in mats]
+    wss = [[T.gemv_workspace(W[c][i], 1) for i in range(len(mats))] for c in range(copies)]
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream(device=dev)
+    launches_per_step = len(mats)
+
+    def step(c):
+        for i in range(len(mats)):
+            T.gemv(W[c][i], xs[i], y=ys[i], workspace=wss[c][i])
+
+    # one CUDA graph per weight copy holds the six launches of a step
+    graphs = []
+    with torch.cuda.stream(stream):
+        for c in range(copies):
+            step(c)  # warm (sets kernel attributes outside capture)
+        torch.cuda.synchronize()
+        for c in range(copies):
+            gph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gph, stream=stream):
+                step(c)
+            graphs.append(gph)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            graphs[i % copies].replay()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(args.steps):
+                graphs[i % copies].replay()
+            e1.record(stream)
+        e1.synchronize()
+    barrier()
+    ms = e0.elapsed_time(e1)
+    ms = max_over_ranks(torch, ms, world, dev)
+    ms_per_step = ms / args.steps
+    value = set_bytes * args.steps * world / (ms * 1e-3) / 1e9
+
+    # per-kernel launch durations in the same steady state (events around single-kernel graphs)
+    per_kernel = time_kernels(torch, T, W, xs, ys, wss, mats, copies, stream)
+    dom = max(per_kernel, key=lambda r: r["ms_total"])
+    achieved = dom["bytes"] / (dom["ms_avg"] * 1e-3) / 1e9
+    traffic = profiled_traffic(dom["key"])
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+                "kernel": dom["key"], "peak_source": peaks["source"] + " hbm_gbs (copy, burst)",
+                "per_kernel": [{k: (round(v, 5) if isinstance(v, float) else v) for k, v in r.items()}
+                               for r in per_kernel]}
+
+    e2e = measure_e2e(torch, T, W, mats, copies, args, stream, world, dev, set_bytes)
+    extras = {} if args.no_extras else measure_extras(torch, T, dev, peaks, stream)
+    cpu = cpu_baseline(torch, T, W, xs, mats) if (rank == 0 and world == 1) else None
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f16 (ternary codes, fp32 accumulate)",
+                "data": "synthetic (seeded codes P(0)=0.4, scales |N(0,1)|*0.02 fp16, x N(0,1) fp16)",
+                "config": {"workload": WORKLOAD, "batch": 1, "layouts": ["Q2_0_g128", "T3_5PB_g128"],
+                           "gemvs_per_step": launches_per_step, "bytes_per_step": set_bytes,
+                           "l2": f"rotating {copies} weight copies ({copies * weight_bytes / 1e6:.0f} MB > 3x L2 "
+                                 f"{l2 / 1e6:.0f} MB)", "parallelism": f"replicas x{world}",
+                           "hbm_frac_of_8TBps": round(value / world / 8000.0, 4)},
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary()}
+        if extras:
+            line["rows"] = extras
+        print(json.dumps(line), flush=True)
+
+
+def max_over_ranks(torch, v, world, dev):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_kernels(torch, T, W, xs, ys, wss, mats, copies, stream, reps=40):
+    """Average device time per launch of each GEMV, replaying a graph of `reps` launches that rotates
+    over the weight copies (HBM-cold weights), timed with CUDA events on the launching stream."""
+    out = []
+    for i, (layout, n, k) in enumerate(mats):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for r in range(reps):
+                    c = r % copies
+                    T.gemv(W[c][i], xs[i], y=ys[i], workspace=wss[c][i])
+            g.replay()
+            torch.cuda.synchronize()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(5):
+                g.replay()
+            b.record(stream)
+        b.synchronize()
+        ms = a.elapsed_time(b) / (5 * reps)
+        nb = algorithmic_bytes(layout, n, k, 1)
+        out.append({"key": f"gemv_{'q2' if layout == T.Q2_0_G128 else 't3'}_{n}x{k}_b1", "bytes": nb,
+                    "ms_avg": ms, "gbs": nb / (ms * 1e-3) / 1e9, "ms_total": ms})
+    return out
+
+
+def measure_e2e(torch, T, W, mats, copies, args, stream, world, dev, set_bytes):
+    """Same step through the public API with host-resident activations: per GEMV, H2D of x from
+    pinned memory, tern_gemv, D2H of y to pinned memory; all inside the event-timed region."""
+    hx = [torch.randn((1, k)).to(torch.float16).pin_memory() for (_, _, k) in mats]
+    hy = [torch.empty((1, n), dtype=torch.float16).pin_memory() for (_, n, _) in mats]
+    dx = [torch.empty((1, k), dtype=torch.float16, device=dev) for (_, _, k) in mats]
+    dy = [torch.empty((1, n), dtype=torch.float16, device=dev) for (_, n, _) in mats]
+    wss = [[T.gemv_workspace(W[c][i], 1) for i in range(len(mats))] for c in range(copies)]
+    steps = max(1, min(args.steps, 500))
+
+    def one(c):
+        for i in range(len(mats)):
+            dx[i].copy_(hx[i], non_blocking=True)
+            T.gemv(W[c][i], dx[i], y=dy[i], workspace=wss[c][i])
+            hy[i].copy_(dy[i], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(min(10, steps)):
+            one(i % copies)
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(steps):
+            one(i % copies)
+        b.record(stream)
+    b.synchronize()
+    ms = max_over_ranks(torch, a.elapsed_time(b), world, dev)
+    h2d = sum(t.numel() * 2 for t in hx)
+    d2h = sum(t.numel() * 2 for t in hy)
+    return {"value": round(set_bytes * steps * world / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(ms / steps, 6), "path": "python binding -> tern_gemv C ABI, eager launches"}
+
+
+def measure_extras(torch, T, dev, peaks, stream):
+    """One line per other row of the hot path: pack, LM head, 27B batched GEMV, prefill GEMM."""
+    res = {}
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def timed(fn, reps):
+        with torch.cuda.stream(stream):
+            fn()
+            torch.cuda.synchronize()
+            a, b = ev(), ev()
+            a.record(stream)
+            for _ in range(reps):
+                fn()
+            b.record(stream)
+        b.synchronize()
+        return a.elapsed_time(b) / reps
+
+    # ternarize + pack of fp16 latents, 8B shapes (both layouts)
+    for layout, name in ((T.Q2_0_G128, "q2"), (T.T3_5PB_G128, "t3")):
+        tot_b, tot_ms = 0, 0.0
+        for (n, k) in LAYER_SET:
+            w = torch.randn((n, k), device=dev).mul_(0.02).to(torch.float16)
+            s = (torch.randn((n, k // GROUP), device=dev).abs() * 0.02).to(torch.float16)
+            Wp = T.pack(w, s, layout)
+            ms = timed(lambda: T.pack(w, s, layout, out=Wp), 20)
+            tot_b += n * k * 2 + n * (k // GROUP) * 2 + n * T.row_bytes(layout, k)
+            tot_ms += ms
+            del w, s, Wp
+        gbs = tot_b / (tot_ms * 1e-3) / 1e9
+        res[f"pack_{name}_8b_set"] = {"GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                                      "ms": round(tot_ms, 5)}
+
+    # LM head (base-3) and 27B batched GEMVs; weights larger than L2, re-read each launch
+    cases = [("lm_head_t3", T.T3_5PB_G128, 151936, 4096, b) for b in (1, 8)]
+    for layout, lname in ((T.Q2_0_G128, "q2"), (T.T3_5PB_G128, "t3")):
+        for (n, k) in ((34816, 5120), (5120, 17408)):
+            for b in (1, 4, 16, 64):
+                cases.append((f"27b_{lname}_{n}x{k}", layout, n, k, b))
+    cache = {}
+    for name, layout, n, k, b in cases:
+        key = (layout, n, k)
+        if key not in cache:
+            cache.clear()
+            torch.cuda.empty_cache()
+            cache[key] = [make_weights(torch, T, n, k, layout, 77 + c, dev) for c in range(2 if n * k > 1e8 else 6)]
+        Ws = cache[key]
+        x = torch.randn((b, k), device=dev).to(torch.float16)
+        y = torch.empty((b, n), dtype=torch.float16, device=dev)
+        wss = [T.gemv_workspace(Wc, b) for Wc in Ws]
+        it = [0]
+
+        def f():
+            c = it[0] % len(Ws)
+            it[0] += 1
+            T.gemv(Ws[c], x, y=y, workspace=wss[c])
+        ms = timed(f, 20)
+        nb = algorithmic_bytes(layout, n, k, b)
+        flops = 2.0 * n * k * b
+        res[f"{name}_b{b}"] = {"GB/s": round(nb / (ms * 1e-3) / 1e9, 1),
+                               "frac_hbm": round(nb / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                               "TFLOP/s": round(flops / (ms * 1e-3) / 1e12, 2), "us": round(ms * 1e3, 2)}
+    cache.clear()
+    torch.cuda.empty_cache()
+
+    # prefill GEMM M=2048, K=5120, N=17408 (Q2_0_g128) on tcgen05
+    try:
+        M, N, K = 2048, 17408, 5120
+        Wg = make_weights(torch, T, N, K, T.Q2_0_G128, 5, dev)
+        X = torch.randn((M, K), device=dev).to(torch.float16)
+        Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        ms = timed(lambda: T.gemm(Wg, X, Y=Y), 20)
+        tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+        res["gemm_q2_2048x17408x5120"] = {"TFLOP/s": round(tf, 1),
+                                          "frac_fp16_peak": round(tf / peaks["bf16_tflops"], 4),
+                                          "peak_TFLOP/s": peaks["bf16_tflops"], "ms": round(ms, 4)}
+    except Exception as e:  # the GEMM is reported, not required for the GEMV metric
+        res["gemm_q2_2048x17408x5120"] = {"error": str(e)[:200]}
+    return res
+
+
+def cpu_baseline(torch, T, W, xs, mats, rows=1024):
+    """The oracle, as it stands, on a bounded sample: `rows` rows of each of the six GEMVs."""
+    import numpy as np
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_limits
+    except Exception:  # pragma: no cover
+        threadpool_limits = None
+    samples = []
+    nbytes = 0
+    for i, (layout, n, k) in enumerate(mats):
+        Wm = W[0][i]
+        r = np.arange(min(rows, n))
+        codes = Wm.codes[: len(r)].cpu().numpy()
+        sc = Wm.scales[: len(r), : k // GROUP].cpu().numpy()
+        x = xs[i].cpu().numpy()
+        samples.append((codes, sc, x, layout, k))
+        nbytes += algorithmic_bytes(layout, len(r), k, 1)
+    ctx = threadpool_limits(limits=1) if threadpool_limits else None
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        for (codes, sc, x, layout, k) in samples:
+            O.gemv(codes, sc, x, layout, k)
+        reps += 1
+        if time.perf_counter() - t0 > 10.0 or reps >= 50:
+            break
+    dt = time.perf_counter() - t0
+    if ctx is not None:
+        ctx.unregister() if hasattr(ctx, "unregister") else None
+    return {"value": round(nbytes * reps / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {rows} rows of each of the six GEMVs x {reps} passes ({dt:.1f} s, numpy fp64, 1 thread)"}
+
+
+# -------------------------------------------------------------------------- the reference arm
+def run_reference(args, rank, world):
+    """The CPU oracle timed on the host cores on a bounded sample of the same workload."""
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle as O
+    from gemm_tern_gemv_b200 import synth
+    try:
+        from threadpoolctl import threadpool_limits
+        lim = threadpool_limits(limits=1)
+    except Exception:
+        lim = None
+    rows = 256
+    samples, nbytes = [], 0
+    for li, layout in enumerate((O.Q2_0_G128, O.T3_5PB_G128)):
+        for mi, (n, k) in enumerate(LAYER_SET):
+            seed = synth.seed_for(2, mi) + 10 * layout
+            t = synth.ternary_codes(rows, k, seed)
+            s = synth.group_scales(rows, k // GROUP, seed)
+            x = synth.activations(1, k, seed)
+            samples.append((O.pack(t, layout), s, x, layout, k))
+            nbytes += rows * O.row_bytes(layout, k) + rows * (k // GROUP) * 2 + 2 * k + 2 * rows
+
+    def step():
+        for (codes, s, x, layout, k) in samples:
+            O.gemv(codes, s, x, layout, k)
+    for _ in range(max(0, args.warmup)):
+        step()
+    steps = max(1, args.steps)
+    t0 = time.perf_counter()
+    done = 0
+    for _ in range(steps):
+        step()
+        done += 1
+        if time.perf_counter() - t0 > 120.0:
+            break
+    dt = time.perf_counter() - t0
+    v = nbytes * done / dt / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": done, "warmup": args.warmup, "ms_per_step": round(dt / done * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded, same distributions)",
+            "config": {"workload": WORKLOAD, "batch": 1, "sample_rows_per_matrix": rows},
+            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{rows} rows of each of the six GEMVs per step (numpy fp64, 1 thread)"},
+            "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = _env_int("WORLD_SIZE", 1)
+    rank = _env_int("RANK", 0)
+    local_rank = _env_int("LOCAL_RANK", 0)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_native(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

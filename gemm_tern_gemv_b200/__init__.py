@@ -1,0 +1,240 @@
+"""Python binding of libtern.so: ternary group-scaled GEMV / GEMM / pack / unpack on B200.
+
+Argument marshalling only. Every step of the computation runs in the library's CUDA kernels;
+PyTorch supplies device memory and the current CUDA stream. There is no fallback: if libtern.so
+is missing or cannot be loaded, every call raises.
+
+    W = pack(w_fp16, scales_fp16, layout=Q2_0_G128)     # ternarize + pack on the GPU
+    y = gemv(W, x)                                       # x [batch][K] fp16 -> y [batch][N] fp16
+    Y = gemm(W, X)                                       # X [M][K] fp16 -> Y [M][N] fp16
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+Q2_0_G128 = 1
+T3_5PB_G128 = 2
+GROUP = 128
+GEMV_MAX_BATCH = 64
+DEVICE_TIMEOUT = 1
+
+STATUS = {0: "TERN_OK", 1: "TERN_ERR_INVALID_ARG", 2: "TERN_ERR_UNSUPPORTED", 3: "TERN_ERR_ALIGNMENT",
+          4: "TERN_ERR_WORKSPACE", 5: "TERN_ERR_INVALID_CODE", 6: "TERN_ERR_TIMEOUT", 7: "TERN_ERR_CUDA"}
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libtern.so")
+
+
+class TernError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({_status_string(status)})")
+
+
+class TernMatrixC(ctypes.Structure):
+    _fields_ = [("layout", ctypes.c_int32), ("n", ctypes.c_int64), ("k", ctypes.c_int64),
+                ("codes", ctypes.c_void_p), ("code_row_stride", ctypes.c_int64),
+                ("scales", ctypes.c_void_p), ("scale_row_stride", ctypes.c_int64)]
+
+
+_lib = None
+
+# name -> (restype, argtypes)
+SIGNATURES = {
+    "tern_row_bytes": (ctypes.c_int64, [ctypes.c_int32, ctypes.c_int64]),
+    "tern_packed_bytes": (ctypes.c_int64, [ctypes.c_int32, ctypes.c_int64, ctypes.c_int64]),
+    "tern_bits_per_weight": (ctypes.c_double, [ctypes.c_int32, ctypes.c_int64]),
+    "tern_pack": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64,
+                                 ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]),
+    "tern_unpack": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                   ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]),
+    "tern_gemv_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(TernMatrixC), ctypes.c_int64]),
+    "tern_gemv": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                 ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "tern_gemm": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                 ctypes.c_void_p, ctypes.c_void_p]),
+    "tern_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "tern_version": (ctypes.c_int32, []),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libtern.so (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m gemm_tern_gemv_b200.build`")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(l, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = l
+    return _lib
+
+
+def _status_string(status: int) -> str:
+    try:
+        return lib().tern_status_string(status).decode()
+    except Exception:  # pragma: no cover - only used while formatting an error
+        return "?"
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise TernError(status, what)
+
+
+def row_bytes(layout: int, k: int) -> int:
+    return int(lib().tern_row_bytes(layout, k))
+
+
+def packed_bytes(layout: int, n: int, k: int) -> int:
+    return int(lib().tern_packed_bytes(layout, n, k))
+
+
+def bits_per_weight(layout: int, k: int) -> float:
+    return float(lib().tern_bits_per_weight(layout, k))
+
+
+def version() -> int:
+    return int(lib().tern_version())
+
+
+# ------------------------------------------------------------------------------- torch plumbing
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_handle():
+    torch = _torch()
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def scale_stride(k: int) -> int:
+    """Row stride (in halves) used for scale tensors: k/128 rounded up to a multiple of 8."""
+    g = k // GROUP
+    return (g + 7) // 8 * 8
+
+
+@dataclass
+class TernMatrix:
+    """A packed ternary matrix on the GPU: codes uint8 [n][code_row_stride], scales fp16 [n][>=k/128]."""
+    layout: int
+    n: int
+    k: int
+    codes: "object"   # torch.uint8 cuda tensor [n][stride]
+    scales: "object"  # torch.float16 cuda tensor [n][sstride]
+
+    def c(self) -> TernMatrixC:
+        return TernMatrixC(self.layout, self.n, self.k, self.codes.data_ptr(), self.codes.stride(0),
+                           self.scales.data_ptr(), self.scales.stride(0))
+
+    @property
+    def nbytes(self) -> int:
+        """Algorithmic bytes of the packed weights: code rows + k/128 scales per row."""
+        return self.n * row_bytes(self.layout, self.k) + self.n * (self.k // GROUP) * 2
+
+
+def empty_matrix(layout: int, n: int, k: int, device="cuda") -> TernMatrix:
+    torch = _torch()
+    codes = torch.empty((n, row_bytes(layout, k)), dtype=torch.uint8, device=device)
+    scales = torch.zeros((n, scale_stride(k)), dtype=torch.float16, device=device)
+    return TernMatrix(layout, n, k, codes, scales)
+
+
+def as_scales(scales, k: int):
+    """fp16 cuda tensor [n][k/128] -> a [n][scale_stride(k)] tensor with 16-byte aligned rows."""
+    torch = _torch()
+    g = k // GROUP
+    if scales.stride(0) % 8 == 0 and scales.stride(1) == 1 and scales.shape[1] >= g and scales.data_ptr() % 16 == 0:
+        return scales
+    out = torch.zeros((scales.shape[0], scale_stride(k)), dtype=torch.float16, device=scales.device)
+    out[:, :g] = scales[:, :g]
+    return out
+
+
+def pack(w, scales, layout: int = Q2_0_G128, out: TernMatrix | None = None) -> TernMatrix:
+    """Ternarize fp16 latents w [n][k] with their group scales [n][k/128] and pack them (tern_pack).
+
+    The returned matrix holds the codes and (a 16-byte-row-aligned copy of) the scales."""
+    torch = _torch()
+    n, k = w.shape
+    scales = as_scales(scales, k)
+    if out is None:
+        codes = torch.empty((n, row_bytes(layout, k)), dtype=torch.uint8, device=w.device)
+        out = TernMatrix(layout, n, k, codes, scales)
+    st = lib().tern_pack(layout, n, k, _ptr(w), w.stride(0), _ptr(scales), scales.stride(0), _ptr(out.codes),
+                         out.codes.stride(0), _stream_handle())
+    _check(st, "tern_pack")
+    return out
+
+
+def from_packed(codes, scales, layout: int, k: int) -> TernMatrix:
+    """Wrap already-packed codes (uint8 [n][>=row_bytes]) and scales as a TernMatrix (device copies)."""
+    torch = _torch()
+    n = codes.shape[0]
+    return TernMatrix(layout, n, k, codes.contiguous(), as_scales(scales, k).contiguous())
+
+
+def unpack(W: TernMatrix, want_w: bool = True, want_t: bool = True):
+    """(w fp16 [n][k] = s*t, t int8 [n][k], invalid-code count) — test/debug path."""
+    torch = _torch()
+    dev = W.codes.device
+    w = torch.empty((W.n, W.k), dtype=torch.float16, device=dev) if want_w else None
+    t = torch.empty((W.n, W.k), dtype=torch.int8, device=dev) if want_t else None
+    cnt = torch.zeros(1, dtype=torch.int32, device=dev)
+    c = W.c()
+    st = lib().tern_unpack(ctypes.byref(c), _ptr(w), W.k, _ptr(t), W.k, _ptr(cnt), _stream_handle())
+    _check(st, "tern_unpack")
+    return w, t, cnt
+
+
+def gemv_workspace_bytes(W: TernMatrix, batch: int) -> int:
+    c = W.c()
+    return int(lib().tern_gemv_workspace_bytes(ctypes.byref(c), batch))
+
+
+def gemv_workspace(W: TernMatrix, batch: int):
+    """A zero-initialised workspace tensor suitable for gemv(W, x) with this batch (or None)."""
+    torch = _torch()
+    nb = gemv_workspace_bytes(W, batch)
+    return torch.zeros(nb, dtype=torch.uint8, device=W.codes.device) if nb else None
+
+
+def gemv(W: TernMatrix, x, y=None, workspace=None):
+    """y [batch][n] = x [batch][k] @ W^T with W ternary (tern_gemv)."""
+    torch = _torch()
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    batch = x.shape[0]
+    x = x.contiguous()
+    if y is None:
+        y = torch.empty((batch, W.n), dtype=torch.float16, device=x.device)
+    if workspace is None:
+        workspace = gemv_workspace(W, batch)
+    wsb = workspace.numel() if workspace is not None else 0
+    c = W.c()
+    st = lib().tern_gemv(ctypes.byref(c), _ptr(x), batch, _ptr(y), _ptr(workspace), wsb, _stream_handle())
+    _check(st, "tern_gemv")
+    return y
+
+
+def gemm(W: TernMatrix, X, Y=None, status=None):
+    """Y [m][n] = X [m][k] @ W^T on tcgen05 tensor cores (tern_gemm)."""
+    torch = _torch()
+    X = X.contiguous()
+    m = X.shape[0]
+    if Y is None:
+        Y = torch.empty((m, W.n), dtype=torch.float16, device=X.device)
+    c = W.c()
+    st = lib().tern_gemm(ctypes.byref(c), _ptr(X), m, _ptr(Y), _ptr(status), _stream_handle())
+    _check(st, "tern_gemm")
+    return Y

@@ -1,0 +1,153 @@
+// C ABI entry points: argument validation, size arithmetic and dispatch to the kernels.
+// Every argument check runs on the host before any CUDA call, so a rejected call touches no
+// device state (and works on a machine without a GPU).
+#include <cmath>
+#include <mutex>
+#include <vector>
+
+#include "tern_internal.cuh"
+
+namespace tern {
+
+int64_t row_bytes(int32_t layout, int64_t k) {
+  if (k <= 0 || k % kGroup) return -1;
+  int64_t b;
+  if (layout == TERN_Q2_0_G128) b = k / 4;           // 4 two-bit codes per byte
+  else if (layout == TERN_T3_5PB_G128) b = (k + 4) / 5;  // 5 trits per byte
+  else return -1;
+  return (b + 15) / 16 * 16;
+}
+
+int sm_count() {
+  static std::mutex mu;
+  static std::vector<int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev >= (int)cache.size()) cache.resize(dev + 1, 0);
+  if (!cache[dev]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cache[dev] = v;
+  }
+  return cache[dev];
+}
+
+}  // namespace tern
+
+using namespace tern;
+
+static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Checks shared by every call that takes a packed matrix.
+static tern_status check_matrix(const tern_matrix* W) {
+  if (!W) return TERN_ERR_INVALID_ARG;
+  if (W->layout != TERN_Q2_0_G128 && W->layout != TERN_T3_5PB_G128) return TERN_ERR_UNSUPPORTED;
+  if (W->n <= 0 || W->k <= 0 || W->k % kGroup) return TERN_ERR_INVALID_ARG;
+  if (W->n > (int64_t)INT32_MAX || W->k > (int64_t)INT32_MAX / 2) return TERN_ERR_INVALID_ARG;
+  if (!W->codes || !W->scales) return TERN_ERR_INVALID_ARG;
+  if (W->code_row_stride < row_bytes(W->layout, W->k)) return TERN_ERR_INVALID_ARG;
+  if (W->scale_row_stride < W->k / kGroup) return TERN_ERR_INVALID_ARG;
+  if (!aligned16(W->codes) || !aligned16(W->scales)) return TERN_ERR_ALIGNMENT;
+  if (W->code_row_stride % 16 || W->scale_row_stride % 8) return TERN_ERR_ALIGNMENT;
+  return TERN_OK;
+}
+
+static tern_status from_cuda(cudaError_t e) { return e == cudaSuccess ? TERN_OK : TERN_ERR_CUDA; }
+
+extern "C" {
+
+int64_t tern_row_bytes(int32_t layout, int64_t k) { return row_bytes(layout, k); }
+
+int64_t tern_packed_bytes(int32_t layout, int64_t n, int64_t k) {
+  int64_t rb = row_bytes(layout, k);
+  if (rb < 0 || n <= 0) return -1;
+  return n * rb;
+}
+
+double tern_bits_per_weight(int32_t layout, int64_t k) {
+  int64_t rb = row_bytes(layout, k);
+  if (rb < 0) return -1.0;
+  return (double)(rb * 8 + (k / kGroup) * 16) / (double)k;
+}
+
+tern_status tern_pack(int32_t layout, int64_t n, int64_t k, const uint16_t* w, int64_t w_row_stride,
+                      const uint16_t* scales, int64_t scale_row_stride, void* codes,
+                      int64_t code_row_stride, void* stream) {
+  if (layout != TERN_Q2_0_G128 && layout != TERN_T3_5PB_G128) return TERN_ERR_UNSUPPORTED;
+  if (n <= 0 || k <= 0 || k % kGroup || n > (int64_t)INT32_MAX || k > (int64_t)INT32_MAX / 2)
+    return TERN_ERR_INVALID_ARG;
+  if (!w || !scales || !codes) return TERN_ERR_INVALID_ARG;
+  if (w_row_stride < k || scale_row_stride < k / kGroup || code_row_stride < row_bytes(layout, k))
+    return TERN_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(scales) || !aligned16(codes)) return TERN_ERR_ALIGNMENT;
+  if (w_row_stride % 8 || scale_row_stride % 8 || code_row_stride % 16) return TERN_ERR_ALIGNMENT;
+  return from_cuda(launch_pack(layout, n, k, w, w_row_stride, scales, scale_row_stride,
+                               static_cast<uint8_t*>(codes), code_row_stride,
+                               static_cast<cudaStream_t>(stream)));
+}
+
+tern_status tern_unpack(const tern_matrix* W, uint16_t* w_out, int64_t w_row_stride, int8_t* t_out,
+                        int64_t t_row_stride, int32_t* invalid_count, void* stream) {
+  tern_status s = check_matrix(W);
+  if (s != TERN_OK) return s;
+  if (!w_out && !t_out) return TERN_ERR_INVALID_ARG;
+  if (w_out && w_row_stride < W->k) return TERN_ERR_INVALID_ARG;
+  if (t_out && t_row_stride < W->k) return TERN_ERR_INVALID_ARG;
+  if ((w_out && (!aligned16(w_out) || w_row_stride % 8)) || (t_out && (!aligned16(t_out) || t_row_stride % 16)))
+    return TERN_ERR_ALIGNMENT;
+  if (invalid_count && (reinterpret_cast<uintptr_t>(invalid_count) & 3u)) return TERN_ERR_ALIGNMENT;
+  return from_cuda(launch_unpack(*W, w_out, w_row_stride, t_out, t_row_stride, invalid_count,
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+size_t tern_gemv_workspace_bytes(const tern_matrix* W, int64_t batch) {
+  if (!W || W->n <= 0 || W->k <= 0 || W->k % kGroup) return 0;
+  if (W->layout != TERN_Q2_0_G128 && W->layout != TERN_T3_5PB_G128) return 0;
+  if (batch < 1 || batch > TERN_GEMV_MAX_BATCH) return 0;
+  return gemv_plan(W->layout, W->n, W->k, batch, sm_count()).ws_bytes;
+}
+
+tern_status tern_gemv(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  tern_status s = check_matrix(W);
+  if (s != TERN_OK) return s;
+  if (batch < 1 || batch > TERN_GEMV_MAX_BATCH || !x || !y) return TERN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return TERN_ERR_ALIGNMENT;
+  GemvPlan plan = gemv_plan(W->layout, W->n, W->k, batch, sm_count());
+  if (plan.ws_bytes) {
+    if (!workspace || workspace_bytes < plan.ws_bytes) return TERN_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return TERN_ERR_ALIGNMENT;
+  }
+  return from_cuda(launch_gemv(*W, x, (int)batch, y, workspace, plan, static_cast<cudaStream_t>(stream)));
+}
+
+tern_status tern_gemm(const tern_matrix* W, const uint16_t* X, int64_t m, uint16_t* Y,
+                      uint32_t* device_status, void* stream) {
+  tern_status s = check_matrix(W);
+  if (s != TERN_OK) return s;
+  if (W->layout != TERN_Q2_0_G128) return TERN_ERR_UNSUPPORTED;
+  if (m <= 0 || m > (int64_t)INT32_MAX || !X || !Y) return TERN_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Y)) return TERN_ERR_ALIGNMENT;
+  if (W->n % 8) return TERN_ERR_ALIGNMENT;  // Y rows are stored as 16-byte vectors
+  if (device_status && (reinterpret_cast<uintptr_t>(device_status) & 3u)) return TERN_ERR_ALIGNMENT;
+  return from_cuda(launch_gemm(*W, X, m, Y, device_status, static_cast<cudaStream_t>(stream)));
+}
+
+const char* tern_status_string(tern_status status) {
+  switch (status) {
+    case TERN_OK: return "ok";
+    case TERN_ERR_INVALID_ARG: return "invalid argument";
+    case TERN_ERR_UNSUPPORTED: return "unsupported layout or size";
+    case TERN_ERR_ALIGNMENT: return "pointer or stride not 16-byte aligned";
+    case TERN_ERR_WORKSPACE: return "split-K workspace missing or too small";
+    case TERN_ERR_INVALID_CODE: return "invalid packed code";
+    case TERN_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case TERN_ERR_CUDA: return "CUDA runtime error";
+  }
+  return "unknown status";
+}
+
+int32_t tern_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,45 @@
+// Internal declarations shared by the library's translation units (not part of the C ABI).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "tern.h"
+
+namespace tern {
+
+constexpr int kGroup = TERN_GROUP;
+
+// Minimum packed row stride in bytes (see tern_row_bytes); -1 on invalid arguments.
+int64_t row_bytes(int32_t layout, int64_t k);
+
+// Number of streaming multiprocessors of the current device (cached per device).
+int sm_count();
+
+// ---- launchers (arguments already validated by the C ABI layer) ----------------------------
+cudaError_t launch_pack(int32_t layout, int64_t n, int64_t k, const uint16_t* w, int64_t w_stride,
+                        const uint16_t* s, int64_t s_stride, uint8_t* codes, int64_t c_stride,
+                        cudaStream_t st);
+
+cudaError_t launch_unpack(const tern_matrix& W, uint16_t* w_out, int64_t w_stride, int8_t* t_out,
+                          int64_t t_stride, int32_t* invalid_count, cudaStream_t st);
+
+// Split-K plan of the decode GEMV for one (layout, n, k, batch) on a device with `sms` SMs.
+struct GemvPlan {
+  int rows_per_cta;     // output rows one CTA produces
+  int row_blocks;       // ceil(n / rows_per_cta)
+  int splits;           // K slices (1 = no workspace)
+  int groups_per_split; // 128-weight groups per slice (a multiple of 5 for base-3 when splits > 1)
+  size_t ws_partial_bytes;  // fp32 partial sums [splits][batch][n]
+  size_t ws_bytes;          // partials + one int32 counter per row block, rounded to 16
+};
+GemvPlan gemv_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms);
+
+cudaError_t launch_gemv(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y,
+                        void* workspace, const GemvPlan& plan, cudaStream_t st);
+
+cudaError_t launch_gemm(const tern_matrix& W, const uint16_t* X, int64_t m, uint16_t* Y,
+                        uint32_t* device_status, cudaStream_t st);
+
+}  // namespace tern

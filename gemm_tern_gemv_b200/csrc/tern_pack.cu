@@ -1,0 +1,223 @@
+// Ternarize-and-pack and unpack kernels for both packed layouts.
+//
+// Both are HBM-streaming kernels: one thread owns one 16-byte chunk of a packed row (64 weights
+// for Q2_0_g128, 80 for base-3), reads or writes the matching fp16 weights with 16-byte vectors,
+// and the grid is sized in whole waves of the SM count with a grid-stride loop.
+//
+// Ternarize rule (QAT re-ternarize step of "Metal 환경에서 ... Bonsai 8B를 파인튜닝", molayo1419.me,
+// paragraph "그것을 파인튜닝하는 방법"): t = round(clamp(w/s, -1, 1)), ties to even. For fp16 w
+// and s the quotient test |w/s| > 1/2 is exactly 2|w| > |s| in fp32 (both sides are exact), so the
+// kernel never divides: t = sign(w)*sign(s) when 2|w| > |s| and s != 0, else 0. NaN compares false
+// and gives 0; an infinite w with finite non-zero s gives +-1; an infinite s gives 0.
+#include <cuda_fp16.h>
+
+#include "tern_internal.cuh"
+
+namespace tern {
+namespace {
+
+constexpr int kThreads = 256;
+
+// t in {-1, 0, +1} of one weight (as int)
+__device__ __forceinline__ int ternary_value(uint16_t wbits, float s_abs, bool s_neg) {
+  float w = __half2float(__ushort_as_half(wbits));
+  bool big = (2.0f * fabsf(w) > s_abs) && (s_abs != 0.0f);
+  return big ? (((w > 0.0f) != s_neg) ? 1 : -1) : 0;
+}
+
+// ---- Q2_0_g128: chunk = 16 bytes = 64 weights, all inside one 128-weight group -------------
+__global__ void __launch_bounds__(kThreads) pack_q2_kernel(const uint16_t* __restrict__ w, int64_t w_stride,
+                                                           const uint16_t* __restrict__ s, int64_t s_stride,
+                                                           uint8_t* __restrict__ codes, int64_t c_stride,
+                                                           int64_t n, int chunks_per_row) {
+  const int64_t total = n * chunks_per_row;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i / chunks_per_row;
+    const int ch = (int)(i - row * chunks_per_row);
+    const int k0 = ch * 64;
+    const float sv = __half2float(__ushort_as_half(s[row * s_stride + k0 / kGroup]));
+    const float s_abs = fabsf(sv);
+    const bool s_neg = sv < 0.0f;
+    const uint4* src = reinterpret_cast<const uint4*>(w + row * w_stride + k0);
+    uint4 v[8];
+#pragma unroll
+    for (int j = 0; j < 8; j++) v[j] = __ldg(src + j);
+    uint32_t out[4];
+#pragma unroll
+    for (int word = 0; word < 4; word++) {
+      uint32_t acc = 0;
+#pragma unroll
+      for (int h = 0; h < 16; h++) {  // weight 16*word + h
+        const uint4& q = v[(16 * word + h) / 8];
+        const int e = (16 * word + h) % 8;
+        const uint32_t pair = (e / 2 == 0) ? q.x : (e / 2 == 1) ? q.y : (e / 2 == 2) ? q.z : q.w;
+        const uint16_t bits = (e & 1) ? (uint16_t)(pair >> 16) : (uint16_t)(pair & 0xFFFFu);
+        acc |= ((uint32_t)ternary_value(bits, s_abs, s_neg) & 3u) << (2 * h);  // 2-bit two's complement
+      }
+      out[word] = acc;
+    }
+    *reinterpret_cast<uint4*>(codes + row * c_stride + (int64_t)ch * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
+
+// ---- base-3: chunk = 16 bytes = 80 trits; trits at k >= K are c = 1 --------------------------
+__global__ void __launch_bounds__(kThreads) pack_t3_kernel(const uint16_t* __restrict__ w, int64_t w_stride,
+                                                           const uint16_t* __restrict__ s, int64_t s_stride,
+                                                           uint8_t* __restrict__ codes, int64_t c_stride,
+                                                           int64_t n, int k, int chunks_per_row) {
+  const int64_t total = n * chunks_per_row;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i / chunks_per_row;
+    const int ch = (int)(i - row * chunks_per_row);
+    const int k0 = ch * 80;
+    const uint16_t* wr = w + row * w_stride;
+    const uint16_t* sr = s + row * s_stride;
+    uint32_t c[80];
+#pragma unroll
+    for (int j = 0; j < 10; j++) {  // 10 vectors of 8 weights; K % 8 == 0 so a vector is all in or all out
+      const int kv = k0 + 8 * j;
+      if (kv < k) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(wr + kv));
+        const float sv = __half2float(__ushort_as_half(sr[kv / kGroup]));  // 8 | 128: one scale per vector
+        const float s_abs = fabsf(sv);
+        const bool s_neg = sv < 0.0f;
+        const uint32_t pr[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int e = 0; e < 8; e++)
+          c[8 * j + e] = (uint32_t)(ternary_value((e & 1) ? (uint16_t)(pr[e / 2] >> 16) : (uint16_t)(pr[e / 2] & 0xFFFFu), s_abs, s_neg) + 1);  // c = t + 1
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; e++) c[8 * j + e] = 1u;
+      }
+    }
+    uint32_t out[4];
+#pragma unroll
+    for (int word = 0; word < 4; word++) {
+      uint32_t acc = 0;
+#pragma unroll
+      for (int b = 0; b < 4; b++) {
+        const int base = 5 * (4 * word + b);
+        const uint32_t byte = c[base] + 3u * c[base + 1] + 9u * c[base + 2] + 27u * c[base + 3] + 81u * c[base + 4];
+        acc |= byte << (8 * b);
+      }
+      out[word] = acc;
+    }
+    *reinterpret_cast<uint4*>(codes + row * c_stride + (int64_t)ch * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
+
+// ---- unpack --------------------------------------------------------------------------------
+template <int LAYOUT>
+__global__ void __launch_bounds__(kThreads) unpack_kernel(const uint8_t* __restrict__ codes, int64_t c_stride,
+                                                          const uint16_t* __restrict__ s, int64_t s_stride,
+                                                          uint16_t* __restrict__ w_out, int64_t w_stride,
+                                                          int8_t* __restrict__ t_out, int64_t t_stride,
+                                                          int32_t* __restrict__ invalid_count,
+                                                          int64_t n, int k, int chunks_per_row) {
+  constexpr int W = (LAYOUT == TERN_Q2_0_G128) ? 64 : 80;  // weights per 16-byte chunk
+  const int64_t total = n * chunks_per_row;
+  int bad = 0;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i / chunks_per_row;
+    const int ch = (int)(i - row * chunks_per_row);
+    const int k0 = ch * W;
+    const uint4 q = __ldg(reinterpret_cast<const uint4*>(codes + row * c_stride + (int64_t)ch * 16));
+    const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+    int8_t t[W];
+#pragma unroll
+    for (int b = 0; b < 16; b++) {
+      const uint32_t byte = (qw[b / 4] >> (8 * (b % 4))) & 0xFFu;
+      if (LAYOUT == TERN_Q2_0_G128) {
+#pragma unroll
+        for (int f = 0; f < 4; f++) {
+          const uint32_t c = (byte >> (2 * f)) & 3u;  // 2-bit two's complement; 0b10 is invalid
+          const bool inv = (c == 2u);
+          bad += inv;
+          t[4 * b + f] = inv ? 0 : (c == 3u ? (int8_t)-1 : (int8_t)c);
+        }
+      } else {
+        const bool inv = byte > 242u;
+        uint32_t v = byte;
+#pragma unroll
+        for (int f = 0; f < 5; f++) {
+          const uint32_t c = v % 3u;
+          v /= 3u;
+          const int kk = k0 + 5 * b + f;
+          bad += (inv && kk < k);
+          t[5 * b + f] = inv ? 0 : (int8_t)((int)c - 1);
+        }
+      }
+    }
+    // outputs: vectors of 8 (fp16) / 16 (int8) weights; K % 16 == 0 so each vector is all in or out
+#pragma unroll
+    for (int j = 0; j < W / 8; j++) {
+      const int kv = k0 + 8 * j;
+      if (w_out && kv < k) {
+        const float sv = __half2float(__ushort_as_half(s[row * s_stride + kv / kGroup]));
+        uint32_t pr[4];
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+          // s * t is exact in fp16: +-s or 0
+          const __half lo = __float2half_rn(sv * (float)t[8 * j + 2 * e]);
+          const __half hi = __float2half_rn(sv * (float)t[8 * j + 2 * e + 1]);
+          pr[e] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+        }
+        *reinterpret_cast<uint4*>(w_out + row * w_stride + kv) = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < W / 16; j++) {
+      const int kv = k0 + 16 * j;
+      if (t_out && kv < k) {
+        uint32_t pr[4];
+#pragma unroll
+        for (int e = 0; e < 4; e++)
+          pr[e] = (uint32_t)(uint8_t)t[16 * j + 4 * e] | ((uint32_t)(uint8_t)t[16 * j + 4 * e + 1] << 8) |
+                  ((uint32_t)(uint8_t)t[16 * j + 4 * e + 2] << 16) | ((uint32_t)(uint8_t)t[16 * j + 4 * e + 3] << 24);
+        *reinterpret_cast<uint4*>(t_out + row * t_stride + kv) = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+      }
+    }
+  }
+  if (invalid_count) {
+    bad = __reduce_add_sync(0xFFFFFFFFu, bad);
+    if ((threadIdx.x & 31) == 0 && bad) atomicAdd(invalid_count, bad);
+  }
+}
+
+int grid_for(int64_t work) {
+  const int64_t waves = (int64_t)sm_count() * 8;  // 8 resident 256-thread blocks per SM
+  const int64_t blocks = (work + kThreads - 1) / kThreads;
+  return (int)(blocks < waves ? (blocks > 0 ? blocks : 1) : waves);
+}
+
+}  // namespace
+
+cudaError_t launch_pack(int32_t layout, int64_t n, int64_t k, const uint16_t* w, int64_t w_stride,
+                        const uint16_t* s, int64_t s_stride, uint8_t* codes, int64_t c_stride,
+                        cudaStream_t st) {
+  const int chunks = (int)(row_bytes(layout, k) / 16);
+  const int grid = grid_for(n * chunks);
+  if (layout == TERN_Q2_0_G128)
+    pack_q2_kernel<<<grid, kThreads, 0, st>>>(w, w_stride, s, s_stride, codes, c_stride, n, chunks);
+  else
+    pack_t3_kernel<<<grid, kThreads, 0, st>>>(w, w_stride, s, s_stride, codes, c_stride, n, (int)k, chunks);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpack(const tern_matrix& W, uint16_t* w_out, int64_t w_stride, int8_t* t_out,
+                          int64_t t_stride, int32_t* invalid_count, cudaStream_t st) {
+  const int chunks = (int)(row_bytes(W.layout, W.k) / 16);
+  const int grid = grid_for(W.n * chunks);
+  const uint8_t* c = static_cast<const uint8_t*>(W.codes);
+  if (W.layout == TERN_Q2_0_G128)
+    unpack_kernel<TERN_Q2_0_G128><<<grid, kThreads, 0, st>>>(c, W.code_row_stride, W.scales, W.scale_row_stride,
+                                                             w_out, w_stride, t_out, t_stride, invalid_count,
+                                                             W.n, (int)W.k, chunks);
+  else
+    unpack_kernel<TERN_T3_5PB_G128><<<grid, kThreads, 0, st>>>(c, W.code_row_stride, W.scales, W.scale_row_stride,
+                                                               w_out, w_stride, t_out, t_stride, invalid_count,
+                                                               W.n, (int)W.k, chunks);
+  return cudaGetLastError();
+}
+
+}  // namespace tern

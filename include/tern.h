@@ -1,0 +1,178 @@
+/*
+ * tern.h — C ABI of the ternary group-scaled matrix-product library for NVIDIA B200 (sm_100a).
+ *
+ * Weights are ternary codes t in {-1, 0, +1} with one IEEE fp16 scale s per 128 consecutive
+ * weights along K, so w = s * t ("Bonsai 27B와 1비트가 살아남는 법", velog.io, section "포맷의
+ * 정체", eq. w_i = s_g * t_i; "Ternary Bonsai 2 27B, 5.93GB로 줄이고도 FP16 성능의 98.2%를 지킨
+ * 삼진 모델", discuss.pytorch.kr, section "그룹 단위 스케일을 공유하는 삼진 형식"). The product
+ * kernels read the packed codes directly and never materialise fp16 weights in device memory
+ * (same page, section "하이브리드 어텐션을 위한 저비트 커널").
+ *
+ * Packed layouts (the pages name the containers but print no bit layout; these are this
+ * library's definitions):
+ *   TERN_Q2_0_G128   t as a 2-bit two's-complement field (0b00 = 0, 0b01 = +1, 0b11 = -1;
+ *                    0b10 is an invalid code); weight k of a row is in byte k/4 at bits
+ *                    2*(k%4)..2*(k%4)+1. A row is K/4 bytes. 2 + 16/128 = 2.125 bits per weight,
+ *                    the 34-bytes-per-128-weights container of the page above, section "두 가지
+ *                    패킹: PTQ1_0과 PQ2_0". A zero-filled row is an all-zero row.
+ *   TERN_T3_5PB_G128 dense base-3: byte j of a row is sum_{i<5} c_{5j+i} * 3^i, c = t + 1; trits
+ *                    past K are c = 1; the row is padded to a multiple of 16 bytes with bytes of
+ *                    value 121 (five c = 1 trits). About 1.725 bits per weight at K = 5120, a
+ *                    stand-in for the denser PTQ1_0 packing of the same section. A byte > 242
+ *                    is invalid.
+ * Scales are a separate fp16 array s[n][g], g = k / 128, with a row stride in halves.
+ *
+ * Conventions for every call:
+ *   - Memory: every pointer argument named as device memory must be device memory (or managed)
+ *     on the current device; the caller owns all buffers. The library allocates no device memory
+ *     per call. tern_gemm keeps a small host-side cache of TMA descriptors.
+ *   - fp16 values are passed as uint16_t bit patterns (IEEE binary16).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). All device work is enqueued
+ *     on it asynchronously; the call returns before the GPU finishes.
+ *   - Argument errors are detected on the host before any launch and returned synchronously; no
+ *     CUDA call is made in that case. A launch failure returns TERN_ERR_CUDA.
+ *   - Alignment: device pointers must be 16-byte aligned and row strides in bytes multiples of 16
+ *     (code_row_stride, 2*scale_row_stride, 2*w_row_stride); otherwise TERN_ERR_ALIGNMENT.
+ *   - Dense activations and outputs are contiguous row-major: x[batch][K], y[batch][N],
+ *     X[M][K], Y[M][N]; products accumulate in fp32 and round the result to fp16 once.
+ *   - No call validates codes except tern_unpack; products on invalid codes give unspecified
+ *     (finite) values.
+ */
+#ifndef TERN_H
+#define TERN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define TERN_API __attribute__((visibility("default")))
+#else
+#define TERN_API
+#endif
+
+#define TERN_GROUP 128           /* weights per fp16 scale */
+#define TERN_GEMV_MAX_BATCH 64   /* largest batch tern_gemv accepts */
+
+typedef enum tern_status {
+  TERN_OK = 0,
+  TERN_ERR_INVALID_ARG = 1,   /* NULL pointer, non-positive size, K % 128 != 0, stride too small */
+  TERN_ERR_UNSUPPORTED = 2,   /* unknown layout id, or a layout/size this entry point lacks */
+  TERN_ERR_ALIGNMENT = 3,     /* pointer or stride not 16-byte aligned */
+  TERN_ERR_WORKSPACE = 4,     /* split-K workspace missing or smaller than required */
+  TERN_ERR_INVALID_CODE = 5,  /* reserved for callers that turn an invalid-code count into a status */
+  TERN_ERR_TIMEOUT = 6,       /* reserved for callers that turn a device timeout flag into a status */
+  TERN_ERR_CUDA = 7           /* a CUDA runtime call or kernel launch failed */
+} tern_status;
+
+typedef enum tern_layout {
+  TERN_Q2_0_G128 = 1,
+  TERN_T3_5PB_G128 = 2
+} tern_layout;
+
+/* Bits of the device status word that tern_gemm writes (atomic OR) when it is non-NULL. */
+#define TERN_DEVICE_TIMEOUT 1u   /* a pipeline wait exceeded its bound; the tile was abandoned */
+
+/* A packed ternary matrix W[n][k] (n output features, k reduction length). Host struct holding
+ * device pointers; the library reads it during the call only. */
+typedef struct tern_matrix {
+  int32_t layout;                 /* tern_layout */
+  int64_t n;                      /* rows (output features), >= 1 */
+  int64_t k;                      /* reduction length, a positive multiple of 128 */
+  const void* codes;              /* device, uint8 [n][code_row_stride] */
+  int64_t code_row_stride;        /* bytes, >= tern_row_bytes(layout, k), multiple of 16 */
+  const uint16_t* scales;         /* device, fp16 [n][scale_row_stride] */
+  int64_t scale_row_stride;       /* halves, >= k / 128, multiple of 8 */
+} tern_matrix;
+
+/* ---- size arithmetic (host only, no CUDA) ------------------------------------------------ */
+
+/* Minimum packed row stride in bytes: K/4 for Q2_0_g128, ceil(K/5) rounded up to 16 for base-3.
+ * Returns -1 for an unknown layout or K not a positive multiple of 128. */
+TERN_API int64_t tern_row_bytes(int32_t layout, int64_t k);
+
+/* n * tern_row_bytes(layout, k): bytes of packed codes at the minimum stride (scales excluded).
+ * Returns -1 on invalid arguments. */
+TERN_API int64_t tern_packed_bytes(int32_t layout, int64_t n, int64_t k);
+
+/* Stored bits per weight at the minimum stride, counting the fp16 scale per 128 weights:
+ * exactly 2.125 for Q2_0_g128; 1.725 for base-3 at K = 5120 ("두 가지 패킹" section's
+ * containers and the information bound log2(3) + 16/128 of section "그룹 단위 스케일을 공유하는
+ * 삼진 형식", eq. b_eff, bound it from below). Returns -1 on invalid arguments. */
+TERN_API double tern_bits_per_weight(int32_t layout, int64_t k);
+
+/* ---- ternarize + pack --------------------------------------------------------------------- */
+
+/* The QAT re-ternarize-and-repack step ("Metal 환경에서 ... Bonsai 8B를 파인튜닝", molayo1419.me,
+ * paragraph "그것을 파인튜닝하는 방법": ternarize each 128-weight group on every forward pass,
+ * then re-pack to 2 bits): t = round(clamp(w / s, -1, 1)) per weight with its group's scale,
+ * ties |w/s| = 1/2 rounding to even (t = 0); s == 0 or NaN, or w NaN, give t = 0. The result is
+ * bit-identical to that rule evaluated with exact division.
+ *   w       device fp16 [n][w_row_stride] latent weights (first k of each row used)
+ *   scales  device fp16 [n][scale_row_stride]
+ *   codes   device uint8 [n][code_row_stride] output; exactly tern_row_bytes(layout, k) bytes of
+ *           each row are written (padding included), the rest of the stride is left untouched.
+ * Errors: TERN_ERR_INVALID_ARG, TERN_ERR_UNSUPPORTED, TERN_ERR_ALIGNMENT, TERN_ERR_CUDA. */
+TERN_API tern_status tern_pack(int32_t layout, int64_t n, int64_t k,
+                      const uint16_t* w, int64_t w_row_stride,
+                      const uint16_t* scales, int64_t scale_row_stride,
+                      void* codes, int64_t code_row_stride, void* stream);
+
+/* ---- unpack (test / debug path; the products never call it) ------------------------------ */
+
+/* Expands W to dense form. Either output may be NULL, not both.
+ *   w_out          device fp16 [n][w_row_stride]: s * t (exact in fp16), 0 for invalid codes
+ *   t_out          device int8 [n][t_row_stride]: t, 0 for invalid codes (t_row_stride bytes)
+ *   invalid_count  device int32 or NULL: the number of weights with an invalid code is ADDED to
+ *                  *invalid_count (caller zeroes it). An invalid base-3 byte counts once per
+ *                  weight it holds. No trap, no abort. */
+TERN_API tern_status tern_unpack(const tern_matrix* W, uint16_t* w_out, int64_t w_row_stride,
+                        int8_t* t_out, int64_t t_row_stride, int32_t* invalid_count, void* stream);
+
+/* ---- decode GEMV (batch 1..64) -------------------------------------------------------------- */
+
+/* Bytes of split-K workspace tern_gemv needs for this matrix and batch (0 when it needs none).
+ * Depends only on (W->layout, W->n, W->k, batch) and the current device's SM count.
+ * Returns 0 also for invalid arguments (tern_gemv then reports the error). */
+TERN_API size_t tern_gemv_workspace_bytes(const tern_matrix* W, int64_t batch);
+
+/* y[b][n] = sum_g s[n][g] * sum_{k in group g} t[n][k] * x[b][k] for b < batch; fp32
+ * accumulation, fp16 result.
+ *   x          device fp16 [batch][k], contiguous
+ *   y          device fp16 [batch][n], contiguous
+ *   workspace  device, >= tern_gemv_workspace_bytes(W, batch) bytes, 16-byte aligned; may be
+ *              NULL when that size is 0. Its trailing counter words must be zero before the first
+ *              call that uses this workspace (e.g. cudaMemset once); every call leaves them zero
+ *              again. Calls that share a workspace must not overlap on the GPU.
+ * Errors: TERN_ERR_INVALID_ARG (batch outside 1..64, ...), TERN_ERR_UNSUPPORTED,
+ *         TERN_ERR_ALIGNMENT, TERN_ERR_WORKSPACE, TERN_ERR_CUDA. */
+TERN_API tern_status tern_gemv(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---- prefill GEMM on tcgen05 tensor cores --------------------------------------------------- */
+
+/* Y[m][n] = sum_k X[m][k] * s[n][k/128] * t[n][k]; packed tiles are decoded to fp16 s*t (exact)
+ * in shared memory and multiplied on the 5th-generation tensor cores with fp32 accumulation in
+ * tensor memory.
+ *   X              device fp16 [m][k], contiguous;  Y device fp16 [m][n], contiguous
+ *   device_status  device uint32 or NULL: TERN_DEVICE_TIMEOUT is OR-ed in if an internal pipeline
+ *                  wait exceeds its bound (the kernel then abandons its work and exits; Y is
+ *                  incomplete). The caller zeroes it.
+ * Only TERN_Q2_0_G128 is supported (base-3 returns TERN_ERR_UNSUPPORTED).
+ * Errors: TERN_ERR_INVALID_ARG, TERN_ERR_UNSUPPORTED, TERN_ERR_ALIGNMENT, TERN_ERR_CUDA. */
+TERN_API tern_status tern_gemm(const tern_matrix* W, const uint16_t* X, int64_t m, uint16_t* Y,
+                      uint32_t* device_status, void* stream);
+
+/* Static description of a status code (never NULL). */
+TERN_API const char* tern_status_string(tern_status status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+TERN_API int32_t tern_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TERN_H */

@@ -21,9 +21,10 @@ Sources (the ternary Bonsai web pages; section names as printed there):
                consume packed weights and fuse unpack + group scale into the product).
 
 Readings of points the pages leave open (each is stated where it is used):
-  R1  Q2_0_g128 bit layout: code c = t + 1 in {0,1,2} (3 is invalid); weight k of a row sits in
-      byte k/4, bits 2*(k%4)..2*(k%4)+1 (little-endian in k); scales are a separate fp16 array
-      s[n][k/128]. Rows are K/4 bytes (always a multiple of 16 because K % 128 == 0).
+  R1  Q2_0_g128 bit layout: the code is t as a 2-bit two's-complement integer (0b00 = 0,
+      0b01 = +1, 0b11 = -1; 0b10 is invalid); weight k of a row sits in byte k/4, bits
+      2*(k%4)..2*(k%4)+1 (little-endian in k); scales are a separate fp16 array s[n][k/128]. Rows
+      are K/4 bytes (always a multiple of 16 because K % 128 == 0).
   R2  Dense base-3 layout (T3_5PB_g128, 5 trits per byte): byte j of a row holds
       sum_{i<5} c_{5j+i} * 3^i with c = t + 1 (a byte > 242 is invalid); the row is a continuous
       trit stream, trits past K are c = 1 (t = 0), and the row is padded with bytes of value 121
@@ -100,16 +101,16 @@ def pack(t: np.ndarray, layout: int) -> np.ndarray:
     _check(layout, k)
     if t.size and (t.min() < -1 or t.max() > 1):
         raise ValueError("codes must be in {-1, 0, +1}")
-    c = (t.astype(np.int64) + 1)  # R1/R2: c = t + 1
     out = np.zeros((n, row_bytes(layout, k)), dtype=np.uint8)
     if layout == Q2_0_G128:
+        c = t.astype(np.int64) & 3  # R1: 2-bit two's complement
         c4 = c.reshape(n, k // 4, 4)
         byte = c4[:, :, 0] + (c4[:, :, 1] << 2) + (c4[:, :, 2] << 4) + (c4[:, :, 3] << 6)
         out[:, : k // 4] = byte.astype(np.uint8)
     else:
         nb = code_bytes(layout, k)
         cp = np.ones((n, nb * 5), dtype=np.int64)  # trits past K are c = 1
-        cp[:, :k] = c
+        cp[:, :k] = t.astype(np.int64) + 1         # R2: c = t + 1
         c5 = cp.reshape(n, nb, 5)
         byte = sum(c5[:, :, i] * _POW3[i] for i in range(5))
         out[:, :nb] = byte.astype(np.uint8)
@@ -120,8 +121,8 @@ def pack(t: np.ndarray, layout: int) -> np.ndarray:
 def unpack(codes: np.ndarray, layout: int, k: int, rows=None, check: bool = True) -> np.ndarray:
     """Unpack uint8 codes [n][stride] (stride >= row_bytes) to int8 t [len(rows)][k].
 
-    With check=True an invalid code (Q2 field == 3, T3 byte > 242 among the bytes that hold the K
-    codes) raises InvalidCode.
+    With check=True an invalid code (Q2 field == 0b10, T3 byte > 242 among the bytes that hold the
+    K codes) raises InvalidCode.
     """
     codes = np.asarray(codes, dtype=np.uint8)
     _check(layout, k)
@@ -131,16 +132,18 @@ def unpack(codes: np.ndarray, layout: int, k: int, rows=None, check: bool = True
     kk = np.arange(k)
     if layout == Q2_0_G128:
         byte = codes[:, kk // 4].astype(np.int64)
-        c = (byte >> (2 * (kk % 4))) & 3
-        bad = c == 3
+        f = (byte >> (2 * (kk % 4))) & 3
+        bad = f == 2
+        t = np.where(f == 3, -1, f)  # two's complement: 3 -> -1
     else:
         byte = codes[:, kk // 5].astype(np.int64)
         c = (byte // np.array(_POW3)[kk % 5]) % 3
         bad = byte > 242
+        t = c - 1
     if check and bad.any():
         r, col = np.argwhere(bad)[0]
         raise InvalidCode(f"invalid code at row {r}, k {col}")
-    t = (c - 1).astype(np.int8)
+    t = t.astype(np.int8)
     if n == 0:
         t = t.reshape(0, k)
     return t
@@ -151,8 +154,8 @@ def count_invalid(codes: np.ndarray, layout: int, n: int, k: int) -> int:
     codes = np.asarray(codes, dtype=np.uint8)[:n]
     kk = np.arange(k)
     if layout == Q2_0_G128:
-        c = (codes[:, kk // 4].astype(np.int64) >> (2 * (kk % 4))) & 3
-        return int((c == 3).sum())
+        f = (codes[:, kk // 4].astype(np.int64) >> (2 * (kk % 4))) & 3
+        return int((f == 2).sum())
     return int((codes[:, kk // 5] > 242).sum())
 
 

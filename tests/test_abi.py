@@ -1,0 +1,139 @@
+"""The C-ABI library loads, exports every symbol include/tern.h declares, and its host-only logic
+(size arithmetic, status strings, argument validation) behaves as documented. No GPU needed: the
+validation paths return before any launch, and pointer arguments here are never dereferenced."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import gemm_tern_gemv_b200 as T
+import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tern.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gemm_tern_gemv_b200 import build
+    build.build()
+    return T.lib()
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"TERN_API\s+[\w\s\*]+?\b(tern_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("tern_pack", "tern_unpack", "tern_gemv", "tern_gemm", "tern_gemv_workspace_bytes",
+              "tern_row_bytes", "tern_packed_bytes", "tern_bits_per_weight", "tern_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", T.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(tern_\w+)", out))
+    missing = [n for n in _declared() if n not in exported]
+    assert not missing, missing
+    for n in _declared():
+        assert hasattr(lib, n)
+    assert set(T.SIGNATURES) >= set(_declared())
+
+
+def test_size_arithmetic_matches_oracle(lib):
+    for layout in (T.Q2_0_G128, T.T3_5PB_G128):
+        for k in list(range(128, 20000, 128)) + [151936 // 128 * 128]:
+            assert T.row_bytes(layout, k) == O.row_bytes(layout, k)
+            assert T.packed_bytes(layout, 7, k) == O.packed_bytes(layout, 7, k)
+            assert T.bits_per_weight(layout, k) == pytest.approx(O.bits_per_weight(layout, k), abs=0, rel=1e-15)
+    assert T.bits_per_weight(T.Q2_0_G128, 4096) == 2.125
+    assert T.bits_per_weight(T.T3_5PB_G128, 5120) == 1.725
+    assert lib.tern_row_bytes(3, 128) == -1
+    assert lib.tern_row_bytes(1, 100) == -1
+    assert lib.tern_row_bytes(1, 0) == -1
+    assert lib.tern_packed_bytes(1, 0, 128) == -1
+    assert lib.tern_bits_per_weight(9, 128) == -1.0
+
+
+def test_status_strings(lib):
+    for s in range(8):
+        assert lib.tern_status_string(s).decode()
+    assert lib.tern_status_string(0).decode() == "ok"
+    assert lib.tern_status_string(99).decode() == "unknown status"
+
+
+# 16-byte aligned and never dereferenced: every call below is rejected on the host before a launch
+FAKE = 0x7F0000000000
+
+
+def _mat(**kw):
+    d = dict(layout=1, n=64, k=1024, codes=FAKE, code_row_stride=256, scales=FAKE + 4096, scale_row_stride=8)
+    d.update(kw)
+    return T.TernMatrixC(d["layout"], d["n"], d["k"], d["codes"], d["code_row_stride"], d["scales"],
+                         d["scale_row_stride"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(layout=0), 2), (dict(layout=3), 2), (dict(n=0), 1), (dict(k=1000), 1), (dict(k=0), 1),
+    (dict(codes=0), 1), (dict(scales=0), 1), (dict(code_row_stride=128), 1), (dict(scale_row_stride=4), 1),
+    (dict(codes=FAKE + 8), 3), (dict(scales=FAKE + 2), 3), (dict(code_row_stride=264), 3),
+    (dict(scale_row_stride=12), 3),
+])
+def test_gemv_rejects_bad_matrix(lib, kw, status):
+    m = _mat(**kw)
+    st = lib.tern_gemv(ctypes.byref(m), ctypes.c_void_p(FAKE), 1, ctypes.c_void_p(FAKE), None, 0, None)
+    assert st == status
+
+
+def test_gemv_rejects_bad_batch_and_buffers(lib):
+    m = _mat()
+    assert lib.tern_gemv(ctypes.byref(m), ctypes.c_void_p(FAKE), 0, ctypes.c_void_p(FAKE), None, 0, None) == 1
+    assert lib.tern_gemv(ctypes.byref(m), ctypes.c_void_p(FAKE), 65, ctypes.c_void_p(FAKE), None, 0, None) == 1
+    assert lib.tern_gemv(ctypes.byref(m), None, 1, ctypes.c_void_p(FAKE), None, 0, None) == 1
+    assert lib.tern_gemv(ctypes.byref(m), ctypes.c_void_p(FAKE + 2), 1, ctypes.c_void_p(FAKE), None, 0, None) == 3
+    assert lib.tern_gemv(None, ctypes.c_void_p(FAKE), 1, ctypes.c_void_p(FAKE), None, 0, None) == 1
+
+
+def test_gemv_workspace_size_and_rejection(lib):
+    # a narrow matrix needs split-K workspace; too little is refused before any launch
+    m = _mat(n=4096, k=4096, code_row_stride=1024, scale_row_stride=32)
+    need = lib.tern_gemv_workspace_bytes(ctypes.byref(m), 1)
+    assert need > 0 and need % 16 == 0
+    assert lib.tern_gemv(ctypes.byref(m), ctypes.c_void_p(FAKE), 1, ctypes.c_void_p(FAKE), None, 0, None) == 4
+    assert lib.tern_gemv(ctypes.byref(m), ctypes.c_void_p(FAKE), 1, ctypes.c_void_p(FAKE),
+                         ctypes.c_void_p(FAKE), need - 16, None) == 4
+    assert lib.tern_gemv(ctypes.byref(m), ctypes.c_void_p(FAKE), 1, ctypes.c_void_p(FAKE),
+                         ctypes.c_void_p(FAKE + 8), need, None) == 3
+    # a tall matrix needs none
+    big = _mat(n=151936, k=4096, code_row_stride=1024, scale_row_stride=32)
+    assert lib.tern_gemv_workspace_bytes(ctypes.byref(big), 1) == 0
+    assert lib.tern_gemv_workspace_bytes(ctypes.byref(big), 0) == 0
+    assert lib.tern_gemv_workspace_bytes(None, 1) == 0
+
+
+def test_pack_unpack_gemm_reject(lib):
+    P = lambda v: ctypes.c_void_p(v)
+    assert lib.tern_pack(3, 4, 128, P(FAKE), 128, P(FAKE), 8, P(FAKE), 32, None) == 2
+    assert lib.tern_pack(1, 4, 130, P(FAKE), 136, P(FAKE), 8, P(FAKE), 48, None) == 1
+    assert lib.tern_pack(1, 4, 128, P(FAKE), 120, P(FAKE), 8, P(FAKE), 32, None) == 1
+    assert lib.tern_pack(1, 4, 128, P(FAKE + 4), 128, P(FAKE), 8, P(FAKE), 32, None) == 3
+    assert lib.tern_pack(2, 4, 128, P(FAKE), 128, P(FAKE), 8, P(FAKE), 16, None) == 1  # base-3 row needs 32
+    m = _mat()
+    assert lib.tern_unpack(ctypes.byref(m), None, 1024, None, 1024, None, None) == 1
+    assert lib.tern_unpack(ctypes.byref(m), P(FAKE), 1000, None, 0, None, None) == 1
+    assert lib.tern_unpack(ctypes.byref(m), P(FAKE), 1028, None, 0, None, None) == 3
+    t3 = _mat(layout=2, code_row_stride=208)
+    assert lib.tern_gemm(ctypes.byref(t3), P(FAKE), 16, P(FAKE), None, None) == 2
+    assert lib.tern_gemm(ctypes.byref(m), P(FAKE), 0, P(FAKE), None, None) == 1
+    assert lib.tern_gemm(ctypes.byref(_mat(n=60)), P(FAKE), 16, P(FAKE), None, None) == 3
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(T, "_lib", None)
+    monkeypatch.setattr(T, "LIB_PATH", str(tmp_path / "nope.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        T.lib()

@@ -81,13 +81,14 @@ def test_q2_byte_table_exhaustive():
     valid = 0
     for byte in range(256):
         fields = [(byte >> (2 * i)) & 3 for i in range(4)]
-        if 3 in fields:
+        if 2 in fields:
             with pytest.raises(O.InvalidCode):
                 O.unpack(codes[byte : byte + 1], O.Q2_0_G128, 128)
             continue
         valid += 1
         t = O.unpack(codes[byte : byte + 1], O.Q2_0_G128, 128)
-        assert list(t[0, :4]) == [f - 1 for f in fields]
+        # a 2-bit two's-complement field: 0b11 is -1
+        assert list(t[0, :4]) == [f - 4 if f >= 2 else f for f in fields]
         assert O.pack(t, O.Q2_0_G128)[0, 0] == byte
     assert valid == 3**4
 
@@ -282,11 +283,18 @@ def test_tolerance_formula():
 def _q2_pack_msb_first(t, layout):
     """Plausible mistake: first weight in the high bits of the byte."""
     n, k = t.shape
-    c = (t.astype(np.int64) + 1).reshape(n, k // 4, 4)
+    c = (t.astype(np.int64) & 3).reshape(n, k // 4, 4)
     out = np.zeros((n, k // 4), dtype=np.uint8)
     for i in range(4):
         out |= (c[:, :, i] << (6 - 2 * i)).astype(np.uint8)
     return out
+
+
+def _q2_pack_offset(t, layout):
+    """Plausible mistake: offset-binary codes c = t + 1 instead of two's complement."""
+    n, k = t.shape
+    c = (t.astype(np.int64) + 1).reshape(n, k // 4, 4)
+    return sum(c[:, :, i] << (2 * i) for i in range(4)).astype(np.uint8)
 
 
 def _t3_pack_reversed_digits(t, layout):
@@ -331,6 +339,7 @@ def test_planted_mistakes_are_caught():
 
     assert hand_ok(lambda r, _: O.pack(r, O.Q2_0_G128), q2)
     assert not hand_ok(_q2_pack_msb_first, q2)
+    assert not hand_ok(_q2_pack_offset, q2)
     assert hand_ok(lambda r, _: O.pack(r, O.T3_5PB_G128), t3)
     assert not hand_ok(_t3_pack_reversed_digits, t3)
 
