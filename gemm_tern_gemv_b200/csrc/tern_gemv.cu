@@ -76,21 +76,25 @@ __host__ __device__ inline size_t smem_bytes(int layout, int nt, int rt, int gps
 // uses slots s0 = 2*(j % 4) (-> b0) and s0 + 1 (-> b1); slot s holds codes (s, s + 8) (lo, hi).
 template <int NT>
 __device__ void build_fragments(const Args& a, int g0, int ngroups, uint2* frag) {
+  // work item = 8 consecutive codes (one 16-byte vector of x) of one (group, batch row)
   uint16_t* fh = reinterpret_cast<uint16_t*>(frag);
-  const int per_group = NT * 4 * kGroup;  // (batch slot, code) pairs per group
-  for (int e = threadIdx.x; e < ngroups * per_group; e += kThreads) {
-    const int gl = e / per_group;
-    const int rem = e % per_group;
-    const int bb = rem / kGroup, kin = rem % kGroup;
-    const uint16_t v = (bb < a.batch) ? a.x[(int64_t)bb * a.k + (int64_t)(g0 + gl) * kGroup + kin] : (uint16_t)0;
-    const int win = gl / 2, gp = gl % 2;
-    const int jt = bb / 4, bp = bb % 4;
-    const int o = 128 * gp + kin;  // code index within the window
-    const int q = o / 64, r = o % 64;
-    const int word = r / 16, i = r % 16;
-    const int sl = i % 8, h = i / 8;
-    const int j = 4 * word + sl / 2;
-    fh[((((size_t)win * 16 + j) * NT + jt) * 16 + bp * 4 + q) * 4 + (sl & 1) * 2 + h] = v;
+  const int items = ngroups * a.batch * 16;
+  for (int e = threadIdx.x; e < items; e += kThreads) {
+    const int v = e & 15;
+    const int gb = e >> 4;
+    const int bb = gb % a.batch, gl = gb / a.batch;
+    const uint4 xv = *reinterpret_cast<const uint4*>(a.x + (int64_t)bb * a.k + (int64_t)(g0 + gl) * kGroup + 8 * v);
+    const int win = gl >> 1, gp = gl & 1;
+    const int jt = bb >> 2, bp = bb & 3;
+    const int o = 128 * gp + 8 * v;       // first code of the vector within the window
+    const int q = o >> 6, word = (o & 63) >> 4, h = v & 1;
+    uint16_t* base = fh + (((size_t)win * 16 + 4 * word) * NT + jt) * 64 + (bp * 4 + q) * 4 + h;
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+    for (int el = 0; el < 8; el++) {      // code i = 8h + el: slot el, MMA j = 4*word + el/2
+      const uint16_t val = (uint16_t)(xw[el >> 1] >> (16 * (el & 1)));
+      base[(size_t)(el >> 1) * NT * 64 + (el & 1) * 2] = val;
+    }
   }
 }
 
@@ -183,7 +187,7 @@ __device__ __forceinline__ void load_pair_t3(const Args& a, int row_base, int g0
 // 16 MMAs over one pair-window, then the fp32 epilogue that applies the two groups' scales.
 template <int NT, int RT>
 __device__ __forceinline__ void mma_pair(const PairCodesT<RT>& p, const uint2* frag, const uint32_t (&mul)[8], int pw,
-                                         int gh, int g, int q, bool bcol, float (&acc)[RT][NT][2]) {
+                                         int gh, int g, int q, const bool (&bload)[NT], float (&acc)[RT][NT][2]) {
   float d[RT][NT][4];
 #pragma unroll
   for (int rt = 0; rt < RT; rt++)
@@ -214,7 +218,7 @@ __device__ __forceinline__ void mma_pair(const PairCodesT<RT>& p, const uint2* f
 #pragma unroll
       for (int jt = 0; jt < NT; jt++) {
         uint2 b = make_uint2(0u, 0u);
-        if (bcol) b = fr[((size_t)j * NT + jt) * 16];
+        if (bload[jt]) b = fr[((size_t)j * NT + jt) * 16];
 #pragma unroll
         for (int rt = 0; rt < RT; rt++) mma_f16(d[rt][jt], a0[rt], a1[rt], a2[rt], a3[rt], b.x, b.y);
       }
@@ -239,13 +243,14 @@ __device__ __forceinline__ void mma_pair(const PairCodesT<RT>& p, const uint2* f
 template <int LAYOUT, int NT, int RT>
 __global__ void __launch_bounds__(kThreads) gemv_kernel(Args a) {
   extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ int last;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int g = lane / 4, q = lane % 4;
   constexpr int ROWS = kWarps * 16 * RT;
-  const int row_block = blockIdx.x;
   const int split = blockIdx.y;
   const int g0 = split * a.gps;
   const int ngroups = min(a.gps, a.groups - g0);
+  const int row_blocks = (a.n + ROWS - 1) / ROWS;
   // shared-memory carve-up must match smem_bytes(), which the host computes from a.gps
   const int wins = (a.gps + 1) / 2 + (LAYOUT == TERN_T3_5PB_G128 ? a.gps / kT3Window + 1 : 0);
 
@@ -254,6 +259,7 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(Args a) {
   uint32_t* lut = reinterpret_cast<uint32_t*>(extra);
   uint8_t* t3buf = extra + 256 * 4 + (size_t)warp * 16 * RT * kQ2RowStride;
 
+  // ---- once per CTA: the activation fragments of this K slice (and the base-3 table) ----
   if (LAYOUT == TERN_T3_5PB_G128) {
     for (int v = threadIdx.x; v < 256; v += kThreads) {
       uint32_t f = 0, r = v < 243 ? v : 121;  // an invalid byte decodes as five t = 0 trits
@@ -261,60 +267,76 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(Args a) {
       for (int i = 0; i < 5; i++) { f |= (((r % 3u) + 3u) & 3u) << (2 * i); r /= 3u; }  // c-1 as 2-bit two's complement
       lut[v] = f;
     }
-  }
-  // The fragment builder indexes windows of two groups from g0; base-3 windows of five groups are
-  // re-based below so that each 5-group window starts a fresh pair.
-  if (LAYOUT == TERN_Q2_0_G128) {
-    build_fragments<NT>(a, g0, ngroups, frag);
-  } else {
-    // groups of 5-window w5 go to pair-windows 3*w5 + (0,0,1,1,2): build per 5-window
+    // groups of 5-window w5 go to pair-windows 3*w5 + (0,0,1,1,2)
     for (int w5 = 0; w5 * kT3Window < ngroups; w5++) {
       const int gn = min(kT3Window, ngroups - w5 * kT3Window);
       build_fragments<NT>(a, g0 + w5 * kT3Window, gn, frag + (size_t)w5 * 3 * 16 * NT * 16);
     }
+  } else {
+    build_fragments<NT>(a, g0, ngroups, frag);
   }
   __syncthreads();
 
-  const int row_base = row_block * ROWS + warp * 16 * RT;
-  float acc[RT][NT][2];
-#pragma unroll
-  for (int rt = 0; rt < RT; rt++)
-#pragma unroll
-    for (int jt = 0; jt < NT; jt++) acc[rt][jt][0] = acc[rt][jt][1] = 0.f;
-
-  const bool bcol = ((g & 1) == (q >> 1));  // this lane's B column (b' = g/2, g' = g&1) matches its group
   // shift multipliers 2^(14 - 2S), built from a runtime 1 so they stay IMAD operands
   uint32_t mul[8];
 #pragma unroll
   for (int S = 0; S < 8; S++) mul[S] = a.unit << (14 - 2 * S);
-  PairCodesT<RT> cur;
-  if (LAYOUT == TERN_Q2_0_G128) {
-    const int npair = (ngroups + 1) / 2;
-    load_pair_q2<RT>(a, row_base, g0, 0, min(2, ngroups), g, q, cur);
-    for (int pw = 0; pw < npair; pw++) {
-      const int gh = min(2, ngroups - 2 * pw);
-      PairCodesT<RT> nxt;
-      if (pw + 1 < npair) load_pair_q2<RT>(a, row_base, g0, 2 * (pw + 1), min(2, ngroups - 2 * (pw + 1)), g, q, nxt);
-      mma_pair<NT, RT>(cur, frag, mul, pw, gh, g, q, bcol, acc);
-      if (pw + 1 < npair) cur = nxt;
-    }
-  } else {
-    const int n5 = (ngroups + kT3Window - 1) / kT3Window;
-    for (int ow = 0; ow < n5; ow++) {
-      const int gn = min(kT3Window, ngroups - ow * kT3Window);
-      __syncwarp();
-      expand_t3_window(a, row_base, 16 * RT, (g0 + ow * kT3Window) / kT3Window, lane, lut, t3buf);
-      __syncwarp();
-      for (int iw = 0; iw < (gn + 1) / 2; iw++) {
-        const int gh = min(2, gn - 2 * iw);
-        load_pair_t3<RT>(a, row_base, g0, ow * kT3Window + 2 * iw, gh, g, q, t3buf, 2 * iw, cur);
-        mma_pair<NT, RT>(cur, frag, mul, 3 * ow + iw, gh, g, q, bcol, acc);
+  // B column of this lane: (b' = g/2, g' = g&1); it carries data when g' is the lane's group
+  const bool bcol = ((g & 1) == (q >> 1));
+  bool bload[NT];
+#pragma unroll
+  for (int jt = 0; jt < NT; jt++) bload[jt] = bcol && (4 * jt + (g >> 1) < a.batch);
+
+  for (int rb = blockIdx.x; rb < row_blocks; rb += gridDim.x) {
+    const int row_base = rb * ROWS + warp * 16 * RT;
+    float acc[RT][NT][2];
+#pragma unroll
+    for (int rt = 0; rt < RT; rt++)
+#pragma unroll
+      for (int jt = 0; jt < NT; jt++) acc[rt][jt][0] = acc[rt][jt][1] = 0.f;
+
+    PairCodesT<RT> cur;
+    if (LAYOUT == TERN_Q2_0_G128) {
+      const int npair = (ngroups + 1) / 2;
+      load_pair_q2<RT>(a, row_base, g0, 0, min(2, ngroups), g, q, cur);
+      for (int pw = 0; pw < npair; pw++) {
+        const int gh = min(2, ngroups - 2 * pw);
+        PairCodesT<RT> nxt;
+        if (pw + 1 < npair) load_pair_q2<RT>(a, row_base, g0, 2 * (pw + 1), min(2, ngroups - 2 * (pw + 1)), g, q, nxt);
+        mma_pair<NT, RT>(cur, frag, mul, pw, gh, g, q, bload, acc);
+        if (pw + 1 < npair) cur = nxt;
+      }
+    } else {
+      const int n5 = (ngroups + kT3Window - 1) / kT3Window;
+      for (int ow = 0; ow < n5; ow++) {
+        const int gn = min(kT3Window, ngroups - ow * kT3Window);
+        __syncwarp();
+        expand_t3_window(a, row_base, 16 * RT, (g0 + ow * kT3Window) / kT3Window, lane, lut, t3buf);
+        __syncwarp();
+        for (int iw = 0; iw < (gn + 1) / 2; iw++) {
+          const int gh = min(2, gn - 2 * iw);
+          load_pair_t3<RT>(a, row_base, g0, ow * kT3Window + 2 * iw, gh, g, q, t3buf, 2 * iw, cur);
+          mma_pair<NT, RT>(cur, frag, mul, 3 * ow + iw, gh, g, q, bload, acc);
+        }
       }
     }
-  }
 
-  // ---- output: lane (g, q) owns y[4*jt + q][row_base + rt*16 + g + 8*hr] ----
-  if (a.splits == 1) {
+    // ---- output: lane (g, q) owns y[4*jt + q][row_base + rt*16 + g + 8*hr] ----
+    if (a.splits == 1) {
+#pragma unroll
+      for (int rt = 0; rt < RT; rt++)
+#pragma unroll
+        for (int jt = 0; jt < NT; jt++)
+#pragma unroll
+          for (int hr = 0; hr < 2; hr++) {
+            const int row = row_base + rt * 16 + g + 8 * hr;
+            const int b = 4 * jt + q;
+            if (row < a.n && b < a.batch)
+              a.y[(int64_t)b * a.n + row] = __half_as_ushort(__float2half_rn(acc[rt][jt][hr]));
+          }
+      continue;
+    }
+    float* part = a.ws + (size_t)split * a.batch * a.n;
 #pragma unroll
     for (int rt = 0; rt < RT; rt++)
 #pragma unroll
@@ -323,39 +345,28 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(Args a) {
         for (int hr = 0; hr < 2; hr++) {
           const int row = row_base + rt * 16 + g + 8 * hr;
           const int b = 4 * jt + q;
-          if (row < a.n && b < a.batch) a.y[(int64_t)b * a.n + row] = __half_as_ushort(__float2half_rn(acc[rt][jt][hr]));
+          if (row < a.n && b < a.batch) part[(size_t)b * a.n + row] = acc[rt][jt][hr];
         }
-    return;
-  }
-  float* part = a.ws + (size_t)split * a.batch * a.n;
-#pragma unroll
-  for (int rt = 0; rt < RT; rt++)
-#pragma unroll
-    for (int jt = 0; jt < NT; jt++)
-#pragma unroll
-      for (int hr = 0; hr < 2; hr++) {
-        const int row = row_base + rt * 16 + g + 8 * hr;
-        const int b = 4 * jt + q;
-        if (row < a.n && b < a.batch) part[(size_t)b * a.n + row] = acc[rt][jt][hr];
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const int prev = atomicAdd(a.counters + rb, 1);
+      last = (prev == a.splits - 1);
+      if (last) a.counters[rb] = 0;  // ready for the next call
+    }
+    __syncthreads();
+    if (last) {
+      __threadfence();
+      const int r0 = rb * ROWS;
+      const int nrows = min(ROWS, a.n - r0);
+      for (int e = threadIdx.x; e < nrows * a.batch; e += kThreads) {
+        const int b = e / nrows, row = r0 + e % nrows;
+        float v = 0.f;
+        for (int sp = 0; sp < a.splits; sp++) v += __ldcg(a.ws + ((size_t)sp * a.batch + b) * a.n + row);
+        a.y[(int64_t)b * a.n + row] = __half_as_ushort(__float2half_rn(v));
       }
-  __threadfence();
-  __syncthreads();
-  __shared__ int last;
-  if (threadIdx.x == 0) {
-    const int prev = atomicAdd(a.counters + row_block, 1);
-    last = (prev == a.splits - 1);
-    if (last) a.counters[row_block] = 0;  // ready for the next call
-  }
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
-  const int r0 = row_block * ROWS;
-  const int nrows = min(ROWS, a.n - r0);
-  for (int e = threadIdx.x; e < nrows * a.batch; e += kThreads) {
-    const int b = e / nrows, row = r0 + e % nrows;
-    float v = 0.f;
-    for (int s = 0; s < a.splits; s++) v += __ldcg(a.ws + ((size_t)s * a.batch + b) * a.n + row);
-    a.y[(int64_t)b * a.n + row] = __half_as_ushort(__float2half_rn(v));
+    }
+    __syncthreads();
   }
 }
 
@@ -367,7 +378,16 @@ cudaError_t launch_t(const Args& a, int row_blocks, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  dim3 grid(row_blocks, a.splits);
+  // persistent CTAs: one full wave, each walking row blocks of its K slice
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  const int wave = sm_count() * per_sm;
+  int gx = (wave + a.splits - 1) / a.splits;
+  if (gx > row_blocks) gx = row_blocks;
+  if (gx < 1) gx = 1;
+  dim3 grid(gx, a.splits);
   kern<<<grid, kThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
