@@ -51,7 +51,9 @@ def parse():
     p.add_argument("--warmup", type=int, default=50)
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--no-extras", action="store_true", help="skip the per-row measurements of the other kernels")
-    p.add_argument("--profile-step", action="store_true", help="few launches, for an ncu launch list")
+    p.add_argument("--profile", default=None, metavar="CASE",
+                   help="run a few launches of one kernel case for ncu: gemv_{q2|t3}_NxK_bB, gemm_q2_MxNxK, "
+                        "pack_{q2|t3}_NxK")
     return p.parse_args()
 
 
@@ -493,8 +495,44 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_profile_case(case: str, launches: int = 6):
+    """A handful of launches of one kernel, for an ncu capture (no timing claims)."""
+    import torch
+    import gemm_tern_gemv_b200 as T
+    dev = torch.device("cuda", 0)
+    parts = case.split("_")
+    kind, layout = parts[0], (T.Q2_0_G128 if parts[1] == "q2" else T.T3_5PB_G128)
+    if kind == "gemv":
+        n, k = (int(v) for v in parts[2].split("x"))
+        b = int(parts[3][1:])
+        W = make_weights(torch, T, n, k, layout, 1, dev)
+        x = torch.randn((b, k), device=dev).to(torch.float16)
+        ws = T.gemv_workspace(W, b)
+        fn = lambda: T.gemv(W, x, workspace=ws)
+    elif kind == "gemm":
+        m, n, k = (int(v) for v in parts[2].split("x"))
+        W = make_weights(torch, T, n, k, layout, 1, dev)
+        X = torch.randn((m, k), device=dev).to(torch.float16)
+        fn = lambda: T.gemm(W, X)
+    elif kind == "pack":
+        n, k = (int(v) for v in parts[2].split("x"))
+        w = torch.randn((n, k), device=dev).mul_(0.02).to(torch.float16)
+        s = (torch.randn((n, k // GROUP), device=dev).abs() * 0.02).to(torch.float16)
+        Wp = T.pack(w, s, layout)
+        fn = lambda: T.pack(w, s, layout, out=Wp)
+    else:
+        raise SystemExit(f"unknown case {case}")
+    for _ in range(launches):
+        fn()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": case, "launches": launches}))
+
+
 def main():
     args = parse()
+    if args.profile:
+        run_profile_case(args.profile)
+        return
     world = _env_int("WORLD_SIZE", 1)
     rank = _env_int("RANK", 0)
     local_rank = _env_int("LOCAL_RANK", 0)
