@@ -31,6 +31,8 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <mutex>
+#include <vector>
 
 #include "sm100.cuh"
 #include "tern_internal.cuh"
@@ -452,7 +454,9 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(Args a) {
       for (int rt = 0; rt < RT; rt++)
 #pragma unroll
         for (int hr = 0; hr < 2; hr++) cp_async16_u32(is_cdst + coff[rt][hr], rp[rt][hr] + gl0 * 32, rsz[rt][hr] & mine);
-      cp_async16_u32(is_sdst, srow + ((g0 + gl0) & ~7), ssz);
+      // one scale row per lane; with 16-row tiles lanes 16..31 issue nothing (a zero-size copy
+      // would still zero-fill its 16 destination bytes, outside this stage)
+      if (ROWS == 32 || lane < ROWS) cp_async16_u32(is_sdst, srow + ((g0 + gl0) & ~7), ssz);
       is_cdst += kCodeStage;
       is_sdst += kScStage;
       if (is_cdst == cring_u + kStages * kCodeStage) {
