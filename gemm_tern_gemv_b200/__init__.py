@@ -53,6 +53,8 @@ SIGNATURES = {
     "tern_gemv_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(TernMatrixC), ctypes.c_int64]),
     "tern_gemv": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                  ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "tern_gemv_noalloc": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                         ctypes.c_void_p]),
     "tern_gemm": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                  ctypes.c_void_p, ctypes.c_void_p]),
     "tern_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -224,6 +226,21 @@ def gemv(W: TernMatrix, x, y=None, workspace=None):
     c = W.c()
     st = lib().tern_gemv(ctypes.byref(c), _ptr(x), batch, _ptr(y), _ptr(workspace), wsb, _stream_handle())
     _check(st, "tern_gemv")
+    return y
+
+
+def gemv_noalloc(W: TernMatrix, x, y=None):
+    """tern_gemv_noalloc: the GEMV without a caller workspace (split-K scratch in a static device
+    array of the library; calls on one device must not overlap on the GPU)."""
+    torch = _torch()
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    x = x.contiguous()
+    if y is None:
+        y = torch.empty((x.shape[0], W.n), dtype=torch.float16, device=x.device)
+    c = W.c()
+    st = lib().tern_gemv_noalloc(ctypes.byref(c), _ptr(x), x.shape[0], _ptr(y), _stream_handle())
+    _check(st, "tern_gemv_noalloc")
     return y
 
 

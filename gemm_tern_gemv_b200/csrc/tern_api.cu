@@ -122,6 +122,14 @@ tern_status tern_gemv(const tern_matrix* W, const uint16_t* x, int64_t batch, ui
   return from_cuda(launch_gemv(*W, x, (int)batch, y, workspace, plan, static_cast<cudaStream_t>(stream)));
 }
 
+tern_status tern_gemv_noalloc(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y, void* stream) {
+  tern_status s = check_matrix(W);
+  if (s != TERN_OK) return s;
+  if (batch < 1 || batch > TERN_GEMV_MAX_BATCH || !x || !y) return TERN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return TERN_ERR_ALIGNMENT;
+  return gemv_noalloc(*W, x, (int)batch, y, static_cast<cudaStream_t>(stream));
+}
+
 tern_status tern_gemm(const tern_matrix* W, const uint16_t* X, int64_t m, uint16_t* Y,
                       uint32_t* device_status, void* stream) {
   tern_status s = check_matrix(W);

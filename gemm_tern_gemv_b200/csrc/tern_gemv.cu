@@ -662,4 +662,47 @@ cudaError_t launch_gemv(const tern_matrix& W, const uint16_t* x, int batch, uint
   return dispatch<TERN_T3_5PB_G128>(a, gx_hint, st);
 }
 
+// ---- allocation-free variant ---------------------------------------------------------------------
+// Split-K scratch in a file-scope device array, for callers that cannot hand the library device
+// memory. Every GPU that loads the library holds these bytes until the process exits.
+static __device__ __align__(256) unsigned char tern_noalloc_scratch[TERN_GEMV_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of tern_noalloc_scratch on the current device, looked up once per device. In
+// host code the array's name is only a host-side stand-in, so it must never be passed to a kernel.
+cudaError_t noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static std::vector<void*> addr;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev >= (int)addr.size()) addr.resize(dev + 1, nullptr);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, tern_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+tern_status gemv_noalloc(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y, cudaStream_t st) {
+  const GemvPlan plan = gemv_plan(W.layout, W.n, W.k, batch, sm_count());
+  if (plan.ws_bytes > (size_t)TERN_GEMV_NOALLOC_SCRATCH_BYTES) return TERN_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (plan.ws_bytes) {
+    if (noalloc_scratch(&scratch) != cudaSuccess) return TERN_ERR_CUDA;
+    // the arrival counters must start at zero; the array keeps whatever the previous call left
+    const size_t counters = plan.ws_bytes - plan.ws_partial_bytes;
+    if (cudaMemsetAsync(static_cast<uint8_t*>(scratch) + plan.ws_partial_bytes, 0, counters, st) != cudaSuccess)
+      return TERN_ERR_CUDA;
+  }
+  return launch_gemv(W, x, batch, y, scratch, plan, st) == cudaSuccess ? TERN_OK : TERN_ERR_CUDA;
+}
+
 }  // namespace tern

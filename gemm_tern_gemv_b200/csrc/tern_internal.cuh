@@ -39,6 +39,9 @@ GemvPlan gemv_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms)
 cudaError_t launch_gemv(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y,
                         void* workspace, const GemvPlan& plan, cudaStream_t st);
 
+// tern_gemv_noalloc's work after argument checks (scratch in a static device array).
+tern_status gemv_noalloc(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y, cudaStream_t st);
+
 cudaError_t launch_gemm(const tern_matrix& W, const uint16_t* X, int64_t m, uint16_t* Y,
                         uint32_t* device_status, cudaStream_t st);
 

@@ -152,6 +152,31 @@ TERN_API size_t tern_gemv_workspace_bytes(const tern_matrix* W, int64_t batch);
 TERN_API tern_status tern_gemv(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y,
                       void* workspace, size_t workspace_bytes, void* stream);
 
+/* Bytes of device memory tern_gemv_noalloc keeps for its split-K scratch (per GPU, for the
+ * lifetime of the process). */
+#define TERN_GEMV_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* tern_gemv without a caller-provided workspace, for callers that cannot allocate device memory
+ * or hand it to a library: e.g. plugins running inside a host runtime that owns every device
+ * allocation and exposes no allocator to them, or loops where cudaMalloc / cudaFree (which can
+ * synchronize the device) are not allowed. This entry point is an engineering addition; the pages
+ * have no counterpart to it.
+ * Same arguments and result as tern_gemv minus the workspace. The split-K scratch it needs lives in
+ * a static device array of TERN_GEMV_NOALLOC_SCRATCH_BYTES that every GPU loading the library
+ * holds until exit; the call allocates nothing and calls no cudaMalloc / cudaFree.
+ *   - The first call on a device looks up that array's device address (cudaGetSymbolAddress) for
+ *     the current device; make that first call before any stream capture.
+ *   - Each call clears the scratch's arrival counters with a stream-ordered memset.
+ *   - Every call on a device shares the one array: calls that overlap on the GPU (different
+ *     streams without ordering between them) race and give wrong results. Order them.
+ *   - A matrix / batch whose split-K workspace (tern_gemv_workspace_bytes) exceeds
+ *     TERN_GEMV_NOALLOC_SCRATCH_BYTES returns TERN_ERR_WORKSPACE before any launch; batch <= 8
+ *     fits for all matrices up to N = 151936, K = 17408.
+ * Errors: those of tern_gemv, TERN_ERR_WORKSPACE as above, TERN_ERR_CUDA if the address lookup
+ * or the memset fails. */
+TERN_API tern_status tern_gemv_noalloc(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y,
+                                       void* stream);
+
 /* ---- prefill GEMM on tcgen05 tensor cores --------------------------------------------------- */
 
 /* Y[m][n] = sum_k X[m][k] * s[n][k/128] * t[n][k]; packed tiles are decoded to fp16 s*t (exact)
