@@ -20,9 +20,6 @@
 #include <cuda_fp16.h>
 
 #include <cstring>
-#include <map>
-#include <mutex>
-#include <tuple>
 
 #include "sm100.cuh"
 #include "tern_internal.cuh"
@@ -257,68 +254,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
   }
 }
 
-// ---- host: tensor maps (driver entry point fetched through the runtime; cached per operand) ----
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled encode_fn() {
-  static EncodeTiled fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiled>(f);
-  });
-  return fn;
-}
-
-bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
-              uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
-  EncodeTiled enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {row_stride_bytes};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// Small host cache of encoded maps keyed by (pointer, shape); the map only depends on those.
-struct MapCache {
-  std::mutex mu;
-  std::map<std::tuple<const void*, uint64_t, uint64_t, uint64_t, int>, CUtensorMap> maps;
-  bool get(CUtensorMap* out, int kind, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
-           uint64_t stride, uint32_t bi, uint32_t bo, CUtensorMapSwizzle sw) {
-    std::lock_guard<std::mutex> lock(mu);
-    auto key = std::make_tuple(base, inner, outer, stride, kind);
-    auto itr = maps.find(key);
-    if (itr != maps.end()) { *out = itr->second; return true; }
-    if (!make_map(out, dt, base, inner, outer, stride, bi, bo, sw)) return false;
-    if (maps.size() > 4096) maps.clear();
-    maps.emplace(key, *out);
-    return true;
-  }
-};
-MapCache& cache() {
-  static MapCache c;
-  return c;
-}
-
 }  // namespace
 
 cudaError_t launch_gemm(const tern_matrix& W, const uint16_t* X, int64_t m, uint16_t* Y, uint32_t* device_status,
                         cudaStream_t st) {
   CUtensorMap mx, mw;
   const uint64_t k = (uint64_t)W.k, n = (uint64_t)W.n;
-  if (!cache().get(&mx, 0, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, X, k, (uint64_t)m, k * 2, BK, BN,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!tmap_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, X, k, (uint64_t)m, k * 2, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  if (!cache().get(&mw, 1, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.codes, k / 4, n, (uint64_t)W.code_row_stride, BK / 4, BM,
-                   CU_TENSOR_MAP_SWIZZLE_NONE))
+  if (!tmap_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.codes, k / 4, n, (uint64_t)W.code_row_stride, BK / 4, BM,
+               CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   Params p;
   p.m = (int)m;

@@ -5,29 +5,28 @@
 // product reads packed codes and fuses unpack + group scale):
 //     y[b][n] = sum_g s[n][g] * sum_{k in g} t[n][k] * x[b][k]
 //
-// How (B200, sm_100a). Batch-1 decode at HBM rate leaves about 0.7 ALU-pipe instructions per
-// weight (LOP3/SHF/PRMT issue at half rate on this SM, on a different pipe than IMAD), and the
-// weights are streamed once, so the kernel is built around two things:
+// How (B200, sm_100a). The weights are streamed once and every code has to be turned into a tensor-
+// core operand, so the integer decode sets the pace (IMAD and LOP3 each issue at half rate, on two
+// different pipes, and an HMMA with freshly decoded operands barely overlaps them):
 //   * Decode = one IMAD + one LOP3 per two weights. A Q2_0_g128 code is t as a 2-bit two's-
 //     complement field; shifted to bits 14..15 of an fp16 half, the field IS the half's sign bit
 //     and exponent MSB: 0b01 -> +2.0, 0b11 -> -2.0, 0b00 -> 0. So (word << (14 - 2i)) & 0xC000C000
 //     is the tensor-core A fragment (2 t_i, 2 t_{i+8}) exactly. B is the fp16 activation itself;
 //     the MMA accumulates D = 2 sum t x in fp32 and the epilogue applies s/2 per group: no offset,
-//     no cancellation, exact products.
-//   * Memory-level parallelism: every warp owns a ring of cp.async stages (16-byte copies straight
-//     to shared memory, no registers) several windows deep and streams its row tiles through it
-//     continuously, so each SM keeps ~100 KB of codes in flight.
-// Layout of the work:
-//   * The 8 MMA columns carry (batch, group-of-window) pairs: a window is two consecutive 128-
-//     weight groups of a row (64 bytes); each lane owns 16 contiguous bytes of it, and the two
-//     groups' partial sums land in different columns, so each gets its own scale in the fp32
-//     epilogue. Up to 4 batch rows share one m16n8k16 tile; larger batches use more n-tiles.
-//   * Activations are written once per CTA into shared memory in B-fragment order.
-//   * Warps walk 32-row tiles of their CTA's K slice. Narrow matrices split K across CTAs; the last
-//     warp to finish a tile (atomic counter) sums the fp32 partials in slice order (deterministic),
-//     stores fp16 y and resets the counter.
-//   * The base-3 layout streams 5-group windows (128 bytes per row) through the ring and expands
-//     them per warp into the same 2-bit fields through a 256-entry table before the same MMA loop.
+//     no cancellation, exact products. The base-3 layout reaches the same fragments with three
+//     integer operations per pair (see dec_t3_word).
+//   * The 8 MMA columns carry (batch, group-within-window) pairs, so each group's partial sum gets
+//     its own scale in the fp32 epilogue. Activations are laid out once per CTA in fragment order.
+// Two kernels:
+//   * gemv_reg_kernel (Q2_0_g128 batch <= 4, base-3 batch <= 2): one window = 64 code bytes of each
+//     row of a 32-row warp tile; every warp streams its windows through its own ring of TMA boxes
+//     (codes and scales, out-of-range reads zero-filled) and decodes them in registers. The
+//     (tile, window) units of a K slice are split into equal runs, one per warp (stream-K), so every
+//     SM gets the same work whatever the matrix shape; tiles shared by several runs are summed
+//     deterministically by the last run to arrive.
+//   * gemv_kernel (larger batches): per-warp cp.async rings over 32- or 16-row tiles, base-3
+//     windows expanded to 2-bit fields in shared memory first; K is split across CTAs for narrow
+//     matrices, with the same last-arriver reduction.
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -59,6 +58,8 @@ struct Args {
   float* ws;        // [splits][batch][n] fp32 partials
   int* counters;    // one per row tile
   int n, k, batch, groups, gps, splits, tiles;
+  int run;          // register kernel: (tile, window) units per warp run (stream-K)
+  int kmax;         // register kernel: partial-sum slots per tile and slice
   uint32_t unit;    // always 1 (see `mul` in the kernel)
 };
 
@@ -569,6 +570,490 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(Args a) {
   cp_async_wait<0>();
 }
 
+// ---- small batches: both layouts decoded in registers ----------------------------------------------
+// One window = 64 code bytes of every row of a warp tile: 256 weights (two groups) of Q2_0_g128 or
+// 320 weights of the base-3 layout. Lane (g, q) owns bytes [16q, 16q + 16) of rows g and g + 8 of
+// each 16-row tile, decodes them straight into mma.sync A fragments and never writes codes back to
+// shared memory:
+//   * Q2_0_g128: slot S of a 16-code word is (word * 2^(14 - 2S)) & 0xC000C000 (see slot()).
+//   * base-3: bytes (0, 2) and (1, 3) of a word sit in 16-bit lanes V; with c = t + 1 the five digits
+//     come out most significant first from one multiply-add and a chain of "times three" steps:
+//     R = V * 202 + 130 maps each byte v to r = floor(R / 64) in [256 v / 81, 256 (v + 1) / 81), so
+//     bits 14..15 of R hold the leading digit and bits 6..13 the scaled remainder p; R' = 3 p * 64
+//     then yields the next digit the same way. Adding 0xC000 per lane turns the digit c into the
+//     two's-complement field of t = c - 1, i.e. the fp16 +-2 / 0 pattern of slot(). Exhaustively
+//     checked over all byte pairs (the carry one lane passes to the other only touches bits that are
+//     masked or already garbage); an invalid byte (> 242) gives unspecified trits.
+// The MMA columns are (batch, group-within-window) pairs: a base-3 window touches three groups, so a
+// lane's four k-slots may belong to two groups and the activation fragments are stored per column.
+#ifndef TERN_REG_WARPS
+#define TERN_REG_WARPS 8
+#endif
+#ifndef TERN_REG_CTAS_PER_SM
+#define TERN_REG_CTAS_PER_SM 2
+#endif
+constexpr int kSWarps = TERN_REG_WARPS;
+constexpr int kSThreads = kSWarps * 32;
+constexpr int kRegCtasPerSm = TERN_REG_CTAS_PER_SM;
+constexpr int kWinBytes = 64;
+
+template <int LAYOUT> struct Lay;
+template <> struct Lay<TERN_Q2_0_G128> {
+  static constexpr int J = 16;   // MMAs per 16-row tile and window
+  static constexpr int C = 1;    // stored fragment columns per batch row (the lane's group is q / 2)
+  static constexpr int SC = 1;   // 16-byte scale chunks per row and window
+  static constexpr int W = 256;  // weights per row and window
+};
+template <> struct Lay<TERN_T3_5PB_G128> {
+  static constexpr int J = 20;
+  static constexpr int C = 3;
+  static constexpr int SC = 2;
+  static constexpr int W = 320;
+};
+
+__host__ __device__ inline int s_windows(int layout, int ngroups) {
+  return layout == TERN_Q2_0_G128 ? (ngroups + 1) / 2 : (ngroups * kGroup + 319) / 320;
+}
+__host__ __device__ constexpr uint32_t s_frag_window_bytes(int layout, int bs) {
+  return layout == TERN_Q2_0_G128 ? 8u * bs * 1 * 4 * 16 : 10u * bs * 3 * 4 * 16;
+}
+__host__ __device__ constexpr uint32_t s_stage_bytes(int layout, int rt) {
+  return (uint32_t)rt * 16 * (kWinBytes + 16 * (layout == TERN_Q2_0_G128 ? 1 : 2));
+}
+__host__ __device__ inline size_t s_smem_bytes(int layout, int rt, int stages, int gps, int bs) {
+  return (size_t)s_frag_window_bytes(layout, bs) * (s_windows(layout, gps) + 1) +
+         (size_t)kSWarps * stages * (s_stage_bytes(layout, rt) + 8) + 16;  // + full barriers, abort flag
+}
+
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
+  int old;
+  asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+__device__ __forceinline__ uint32_t lds16(uint32_t addr) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+
+// Base-3 word (bytes b0..b3) -> 10 A registers: o[5h + i] = (2 t of digit 4 - i of byte h,
+// same digit of byte 2 + h) as an fp16 pair.
+__device__ __forceinline__ void dec_t3_word(uint32_t w, uint32_t k0, uint32_t (&o)[10]) {
+#pragma unroll
+  for (int h = 0; h < 2; h++) {
+    const uint32_t V = h ? __byte_perm(w, 0u, 0x4341) : (w & 0x00FF00FFu);
+    uint32_t R = V * 202u + k0;
+    o[5 * h] = R & 0xC000C000u;
+    R = (R & 0x3FC03FC0u) * 3u + 0xC000C000u;
+    o[5 * h + 1] = R & 0xC000C000u;
+#pragma unroll
+    for (int i = 2; i < 5; i++) {
+      R = (R - o[5 * h + i - 1]) * 3u + 0xC000C000u;
+      o[5 * h + i] = R & 0xC000C000u;
+    }
+  }
+}
+
+// Activation fragments of one K slice, one entry (uint2 = the lane's b0, b1) per
+// [window][mma j / 2][batch slot][column c < C][q][j % 2], so a lane reads two MMAs' worth with one
+// 16-byte load. Column c is the group within the window (base-3) or implied by q (Q2). One extra
+// window of zeros follows: lanes whose MMA column carries no data read it.
+// Built from (window, lane chunk q, batch row, half) units whose code positions are compile-time.
+template <int LAYOUT, int BS, int HF>
+__device__ __forceinline__ void s_frag_half(const Args& a, int g0, int kslice, int w, int q, int b, uint16_t* fh) {
+  using L = Lay<LAYOUT>;
+  constexpr int HW = L::W / 8;  // weights of a lane chunk half: 32 (Q2) or 40 (base-3)
+  const int k0 = w * L::W + (L::W / 4) * q + HF * HW;  // first weight within the slice
+  const uint16_t* xs = a.x + (int64_t)b * a.k + (int64_t)g0 * kGroup + k0;
+  uint32_t xw[HW / 2];
+#pragma unroll
+  for (int v = 0; v < HW / 8; v++) {
+    uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+    if (k0 + 8 * v < kslice) xv = *reinterpret_cast<const uint4*>(xs + 8 * v);
+    xw[4 * v] = xv.x; xw[4 * v + 1] = xv.y; xw[4 * v + 2] = xv.z; xw[4 * v + 3] = xv.w;
+  }
+  const int colbase = LAYOUT == TERN_Q2_0_G128 ? 0 : 320 * (w & 1) + 80 * q + HF * HW;
+#pragma unroll
+  for (int cc = 0; cc < HW; cc++) {
+    const int c = HF * HW + cc;  // position within the lane's chunk
+    int j, e4, col = 0;
+    if (LAYOUT == TERN_Q2_0_G128) {
+      const int word = c >> 4, i = c & 15, S = i & 7;
+      j = 4 * word + (S >> 1);
+      e4 = 2 * (S & 1) + (i >> 3);
+    } else {
+      const int bl = c / 5, d = c - 5 * bl, word = bl >> 2, bb = bl & 3;
+      const int r = 5 * (bb & 1) + (4 - d);
+      j = 5 * word + (r >> 1);
+      e4 = 2 * (r & 1) + (bb >> 1);
+      col = ((colbase + cc) >> 7) - 2 * (w & 1);
+    }
+    const int entry = (((((w * (L::J / 2) + (j >> 1)) * BS + b) * L::C + col) * 4 + q) * 2 + (j & 1));
+    fh[entry * 4 + e4] = (uint16_t)(xw[cc >> 1] >> (16 * (cc & 1)));
+  }
+}
+
+template <int LAYOUT, int BS>
+__device__ void s_build_frag(const Args& a, int g0, int ngroups, int nwin_alloc, uint8_t* frag) {
+  constexpr uint32_t FW = s_frag_window_bytes(LAYOUT, BS);
+  uint4* f4 = reinterpret_cast<uint4*>(frag);
+  if (LAYOUT == TERN_Q2_0_G128) {
+    // every entry a data lane reads is written below (zero past the slice); only the zero block
+    for (int i = threadIdx.x; i < (int)(FW / 16); i += kSThreads)
+      f4[(size_t)nwin_alloc * FW / 16 + i] = make_uint4(0u, 0u, 0u, 0u);
+  } else {
+    // base-3 entries hold one group column each: the other columns must read as zero
+    for (int i = threadIdx.x; i < (int)((nwin_alloc + 1) * FW / 16); i += kSThreads) f4[i] = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+  }
+  uint16_t* fh = reinterpret_cast<uint16_t*>(frag);
+  const int kslice = ngroups * kGroup;
+  const int nwin = s_windows(LAYOUT, ngroups);
+  const int items = nwin * 4 * a.batch * 2;
+  for (int e = threadIdx.x; e < items; e += kSThreads) {
+    const int hf = e & 1, q = (e >> 1) & 3, rest = e >> 3;
+    const int b = rest % a.batch, w = rest / a.batch;
+    if (hf == 0) s_frag_half<LAYOUT, BS, 0>(a, g0, kslice, w, q, b, fh);
+    else s_frag_half<LAYOUT, BS, 1>(a, g0, kslice, w, q, b, fh);
+  }
+}
+
+// Stream-K bookkeeping of the small-batch kernel. In every K slice the units (tile, window), tile-
+// major, are cut into runs of a.run consecutive units, run i going to warp i of the slice (the last
+// run may be shorter; warps past the last run idle). The runs that touch a tile are consecutive and
+// each writes one partial-sum slot.
+template <int LAYOUT>
+__device__ __forceinline__ int s_nseg(const Args& a, int split, int tile) {  // runs touching a tile in a slice
+  const int ng = min(a.gps, a.groups - split * a.gps);
+  const int nwin = s_windows(LAYOUT, ng);
+  const uint32_t f = (uint32_t)tile * nwin;
+  return (int)((f + nwin - 1) / (uint32_t)a.run - f / (uint32_t)a.run) + 1;
+}
+
+template <int LAYOUT>
+__device__ __forceinline__ int s_contributors(const Args& a, int tile) {  // runs touching a tile, all slices
+  int c = 0;
+  for (int sp = 0; sp < a.splits; sp++) c += s_nseg<LAYOUT>(a, sp, tile);
+  return c;
+}
+
+// Lane (g, q) accumulates rows g, g + 8 of each 16-row tile. Q2: lane q holds batch q. Base-3: lanes
+// q and q ^ 1 hold batch q / 2 (groups 0-1 and 2 of each window) and are summed here; the even lane
+// of the pair stores.
+template <int LAYOUT, int RT>
+__device__ __forceinline__ void s_combine(float (&acc)[RT][2], int& b, bool& owner, int q) {
+  b = q;
+  owner = true;
+  if (LAYOUT == TERN_T3_5PB_G128) {
+#pragma unroll
+    for (int rt = 0; rt < RT; rt++)
+#pragma unroll
+      for (int hr = 0; hr < 2; hr++) acc[rt][hr] += __shfl_xor_sync(0xFFFFFFFFu, acc[rt][hr], 1);
+    b = q >> 1;
+    owner = (q & 1) == 0;
+  }
+}
+
+// y for a tile this run covers alone, or the run's fp32 partial in its (slice, rank) slot.
+template <int LAYOUT, int RT>
+__device__ __forceinline__ void s_store(const Args& a, int tile, int slot, int lane, float (&acc)[RT][2]) {
+  const int g = lane >> 2, q = lane & 3;
+  int b;
+  bool owner;
+  s_combine<LAYOUT, RT>(acc, b, owner, q);
+  const int row_base = tile * 16 * RT;
+  float* part = slot >= 0 ? a.ws + (size_t)slot * a.batch * a.n : nullptr;
+#pragma unroll
+  for (int rt = 0; rt < RT; rt++)
+#pragma unroll
+    for (int hr = 0; hr < 2; hr++) {
+      const int row = row_base + rt * 16 + g + 8 * hr;
+      if (owner && row < a.n && b < a.batch) {
+        if (slot < 0) a.y[(int64_t)b * a.n + row] = __half_as_ushort(__float2half_rn(0.5f * acc[rt][hr]));
+        else part[(size_t)b * a.n + row] = 0.5f * acc[rt][hr];
+      }
+    }
+}
+
+// The last run to arrive at a tile sums every slot in (slice, rank) order (so the result does not
+// depend on timing), stores y and re-arms the tile's counter for the next call.
+template <int LAYOUT, int RT>
+__device__ __forceinline__ void s_reduce_tile(const Args& a, int tile, int lane) {
+  const int row_base = tile * 16 * RT;
+  const int rows = min(16 * RT, a.n - row_base);
+  for (int e = lane; e < rows * a.batch; e += 32) {
+    const int bb = e / rows, row = row_base + e % rows;
+    float v = 0.f;
+    for (int sp = 0; sp < a.splits; sp++) {
+      const int ns = s_nseg<LAYOUT>(a, sp, tile);
+      const float* src = a.ws + ((size_t)(sp * a.kmax) * a.batch + bb) * a.n + row;
+      const size_t slot_stride = (size_t)a.batch * a.n;
+      float pv[4];
+      int k = 0;
+      for (; k + 4 <= ns; k += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; u++) pv[u] = __ldcg(src + (k + u) * slot_stride);
+#pragma unroll
+        for (int u = 0; u < 4; u++) v += pv[u];
+      }
+      for (; k < ns; k++) v += __ldcg(src + k * slot_stride);
+    }
+    a.y[(int64_t)bb * a.n + row] = __half_as_ushort(__float2half_rn(v));
+  }
+  __syncwarp();
+  if (lane == 0) a.counters[tile] = 0;
+}
+
+// Publishes the partial slots a run wrote (at most two tiles: the one it started inside and the one
+// it ended inside) with one fence, then takes part in the arrival count of each; the partial stores
+// and the fence are issued by every lane before lane 0's atomics, and the last arriver fences again
+// before reading the other runs' slots.
+template <int LAYOUT, int RT>
+__device__ __forceinline__ void s_publish(const Args& a, const int (&tile)[2], const int (&contrib)[2], int n, int lane) {
+  __threadfence();
+  __syncwarp();
+  int prev[2] = {0, 0};
+  if (lane == 0) {
+#pragma unroll
+    for (int i = 0; i < 2; i++)
+      if (i < n) prev[i] = atomicAdd(a.counters + tile[i], 1);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; i++) {
+    if (i >= n) break;
+    const int p = __shfl_sync(0xFFFFFFFFu, prev[i], 0);
+    if (p == contrib[i] - 1) {
+      __threadfence();
+      s_reduce_tile<LAYOUT, RT>(a, tile[i], lane);
+    }
+  }
+}
+
+constexpr uint64_t kRegWaitLimitNs = 1000000000ull;  // 1 s: far beyond any healthy TMA latency
+
+template <int LAYOUT, int RT, int BS, int STAGES>
+__global__ void __launch_bounds__(kSThreads, kRegCtasPerSm)
+    gemv_reg_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales, Args a) {
+  using L = Lay<LAYOUT>;
+  constexpr int ROWS = RT * 16;
+  constexpr uint32_t FW = s_frag_window_bytes(LAYOUT, BS);
+  constexpr uint32_t STAGE = s_stage_bytes(LAYOUT, RT);
+  constexpr uint32_t kCodeBytes = ROWS * kWinBytes;
+  constexpr uint32_t kJP = BS * L::C * 64;  // bytes between fragment pairs (j / 2) of one window
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, q = lane & 3;
+  const int split = blockIdx.y;
+  const int g0 = split * a.gps;
+  const int ngroups = min(a.gps, a.groups - g0);
+  const int nwin = s_windows(LAYOUT, ngroups);
+  const int nwin_alloc = s_windows(LAYOUT, a.gps);
+  uint8_t* frag = smem;
+  uint8_t* rings = smem + (size_t)(nwin_alloc + 1) * FW;
+  uint8_t* ring = rings + (size_t)warp * STAGES * STAGE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(rings + (size_t)kSWarps * STAGES * STAGE) + warp * STAGES;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(
+      reinterpret_cast<uint64_t*>(rings + (size_t)kSWarps * STAGES * STAGE) + kSWarps * STAGES);
+
+  if (lane == 0) {
+    for (int s = 0; s < STAGES; s++) sm100::mbar_init(full + s, 1);
+    sm100::fence_mbar_init();
+    sm100::prefetch_tmap(&tm_codes);
+    sm100::prefetch_tmap(&tm_scales);
+  }
+  if (threadIdx.x == 0) *abort_flag = 0;
+  __syncwarp();
+
+  // this warp's run of (tile, window) units in the slice (empty past the last run)
+  const int wi = blockIdx.x * kSWarps + warp;
+  const int units = a.tiles * nwin;
+  const int u_begin = min(wi * a.run, units);
+  const int u_end = min(u_begin + a.run, units);
+  const int total = u_end - u_begin;
+  const int tile0 = u_begin / nwin, w0 = u_begin - tile0 * nwin;
+
+  // ---- issue side (lane 0): one TMA box of codes [ROWS][64 B] and one of scales per window; reads
+  // past the row data, the scale columns or the last row are zero-filled by the tensor maps
+  const int slice_x0 = LAYOUT == TERN_Q2_0_G128 ? g0 * (kGroup / 4) : (g0 / 5) * 128;
+  int is_tile = tile0, is_w = w0, is_slot = 0;
+  auto issue_next = [&]() {
+    uint64_t* bar = full + is_slot;
+    uint8_t* dst = ring + is_slot * STAGE;
+    const int gfirst = LAYOUT == TERN_Q2_0_G128 ? g0 + 2 * is_w : g0 + (5 * is_w) / 2;
+    sm100::mbar_arrive_expect_tx(bar, STAGE);
+    sm100::tma_load_2d(dst, &tm_codes, bar, slice_x0 + kWinBytes * is_w, is_tile * ROWS);
+    sm100::tma_load_2d(dst + kCodeBytes, &tm_scales, bar, 8 * (gfirst >> 3), is_tile * ROWS);
+    if (++is_slot == STAGES) is_slot = 0;
+    if (++is_w == nwin) {
+      is_w = 0;
+      ++is_tile;
+    }
+  };
+  if (lane == 0)
+    for (int st = 0; st < STAGES && st < total; st++) issue_next();
+
+  s_build_frag<LAYOUT, BS>(a, g0, ngroups, nwin_alloc, frag);
+
+  // B column of this lane and the fragment address it reads (zero block when it carries no data)
+  int fb, fcol;
+  bool fdata;
+  if (LAYOUT == TERN_Q2_0_G128) {
+    fb = g >> 1; fcol = 0; fdata = ((g & 1) == (q >> 1)) && fb < a.batch;
+  } else {
+    fb = g >> 2; fcol = g & 3; fdata = fcol < 3 && fb < a.batch;
+  }
+  const uint32_t fbase = fdata ? smem_u32(frag) + ((fb * L::C + fcol) * 4 + q) * 16
+                               : smem_u32(frag) + (uint32_t)nwin_alloc * FW;
+  const uint32_t fstep = fdata ? FW : 0u;
+
+  uint32_t mul[8];
+#pragma unroll
+  for (int S = 0; S < 8; S++) mul[S] = a.unit << (14 - 2 * S);
+  const uint32_t k0 = a.unit * (130u | (130u << 16)) + 0xC000C000u;
+
+  float acc[RT][2];
+#pragma unroll
+  for (int rt = 0; rt < RT; rt++) acc[rt][0] = acc[rt][1] = 0.f;
+
+  __syncthreads();  // fragments and barrier initialisation visible to every warp
+  const uint32_t ring_u = smem_u32(ring);
+  const uint32_t lane_code = (g * kWinBytes) + 16 * q;       // + (rt * 16 + 8 hr) * 64
+  const uint32_t lane_scale = kCodeBytes + g * (16 * L::SC);  // + (rt * 16 + 8 hr) * 16 * SC
+  int c_tile = tile0, c_w = w0, c_slot = 0;
+  int pend_tile[2] = {0, 0}, pend_contrib[2] = {0, 0}, npend = 0;  // partial tiles awaiting their count
+  int st = 0;
+  for (; st < total; st++) {
+    if (!sm100::mbar_wait_bounded(full + c_slot, (st / STAGES) & 1, abort_flag, nullptr, 0u, kRegWaitLimitNs)) break;
+    const uint32_t stage_u = ring_u + c_slot * STAGE;
+    // activation fragments of the window
+    uint4 bfr[L::J / 2];
+    const uint32_t fa = fbase + (uint32_t)c_w * fstep;
+#pragma unroll
+    for (int jp = 0; jp < L::J / 2; jp++) bfr[jp] = lds128(fa + jp * kJP);
+    uint4 cw[RT][2];
+#pragma unroll
+    for (int rt = 0; rt < RT; rt++)
+#pragma unroll
+      for (int hr = 0; hr < 2; hr++) cw[rt][hr] = lds128(stage_u + lane_code + (rt * 16 + 8 * hr) * kWinBytes);
+    // the two scales this lane's columns use, per row (columns without data have D = 0)
+    float sa[RT][2], sb[RT][2];
+    {
+      const int gfirst = LAYOUT == TERN_Q2_0_G128 ? g0 + 2 * c_w : g0 + (5 * c_w) / 2;
+      const int ja = LAYOUT == TERN_Q2_0_G128 ? 0 : 2 * (q & 1);
+      const uint32_t so = stage_u + lane_scale + 2 * ((gfirst & 7) + ja);
+#pragma unroll
+      for (int rt = 0; rt < RT; rt++)
+#pragma unroll
+        for (int hr = 0; hr < 2; hr++) {
+          const uint32_t ra = so + (rt * 16 + 8 * hr) * (16 * L::SC);
+          if (LAYOUT == TERN_Q2_0_G128) {
+            const uint32_t pr = lds32(ra);  // groups gfirst, gfirst + 1 (gfirst is even)
+            const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&pr));
+            sa[rt][hr] = sf.x;
+            sb[rt][hr] = sf.y;
+          } else {
+            sa[rt][hr] = __half2float(__ushort_as_half((unsigned short)lds16(ra)));
+            sb[rt][hr] = __half2float(__ushort_as_half((unsigned short)lds16(ra + 2)));
+          }
+        }
+    }
+    float d[RT][4];
+    if (LAYOUT == TERN_Q2_0_G128) {
+#pragma unroll
+      for (int word = 0; word < 4; word++) {
+        uint32_t wl[RT], wh[RT];
+#pragma unroll
+        for (int rt = 0; rt < RT; rt++) {
+          wl[rt] = word == 0 ? cw[rt][0].x : word == 1 ? cw[rt][0].y : word == 2 ? cw[rt][0].z : cw[rt][0].w;
+          wh[rt] = word == 0 ? cw[rt][1].x : word == 1 ? cw[rt][1].y : word == 2 ? cw[rt][1].z : cw[rt][1].w;
+        }
+#pragma unroll
+        for (int sp = 0; sp < 4; sp++) {
+          const int j = 4 * word + sp;
+          const uint4 bq = bfr[j >> 1];
+          const uint32_t b0 = (j & 1) ? bq.z : bq.x, b1 = (j & 1) ? bq.w : bq.y;
+#pragma unroll
+          for (int rt = 0; rt < RT; rt++) {
+            const uint32_t a0 = slot(wl[rt], mul[2 * sp]), a2 = slot(wl[rt], mul[2 * sp + 1]);
+            const uint32_t a1 = slot(wh[rt], mul[2 * sp]), a3 = slot(wh[rt], mul[2 * sp + 1]);
+            if (j == 0) mma_f16_first(d[rt], a0, a1, a2, a3, b0, b1);
+            else mma_f16(d[rt], a0, a1, a2, a3, b0, b1);
+          }
+        }
+      }
+    } else {
+#pragma unroll
+      for (int word = 0; word < 4; word++) {
+        uint32_t o[RT][2][10];
+#pragma unroll
+        for (int rt = 0; rt < RT; rt++)
+#pragma unroll
+          for (int hr = 0; hr < 2; hr++) {
+            const uint32_t wv = word == 0 ? cw[rt][hr].x : word == 1 ? cw[rt][hr].y : word == 2 ? cw[rt][hr].z : cw[rt][hr].w;
+            dec_t3_word(wv, k0, o[rt][hr]);
+          }
+#pragma unroll
+        for (int m = 0; m < 5; m++) {
+          const int j = 5 * word + m;
+          const uint4 bq = bfr[j >> 1];
+          const uint32_t b0 = (j & 1) ? bq.z : bq.x, b1 = (j & 1) ? bq.w : bq.y;
+#pragma unroll
+          for (int rt = 0; rt < RT; rt++) {
+            if (j == 0) mma_f16_first(d[rt], o[rt][0][2 * m], o[rt][1][2 * m], o[rt][0][2 * m + 1], o[rt][1][2 * m + 1], b0, b1);
+            else mma_f16(d[rt], o[rt][0][2 * m], o[rt][1][2 * m], o[rt][0][2 * m + 1], o[rt][1][2 * m + 1], b0, b1);
+          }
+        }
+      }
+    }
+    // lane (g, q) holds columns 2q, 2q + 1 of rows g (d[0..1]) and g + 8 (d[2..3]); D = 2 sum t x
+#pragma unroll
+    for (int rt = 0; rt < RT; rt++)
+#pragma unroll
+      for (int hr = 0; hr < 2; hr++)
+        acc[rt][hr] = fmaf(sb[rt][hr], d[rt][2 * hr + 1], fmaf(sa[rt][hr], d[rt][2 * hr], acc[rt][hr]));
+    // every lane has read this stage: refill it with the window STAGES ahead
+    __syncwarp();
+    if (lane == 0 && st + STAGES < total) issue_next();
+    if (++c_slot == STAGES) c_slot = 0;
+    if (++c_w == nwin || st == total - 1) {
+      // end of this warp's run inside the tile: a tile covered by this run alone gets y now; a shared
+      // one gets this run's partial in the slot of its rank among the tile's runs
+      const int contributors = s_contributors<LAYOUT>(a, c_tile);
+      if (contributors == 1) {
+        s_store<LAYOUT, RT>(a, c_tile, -1, lane, acc);
+      } else {
+        const int seg = wi - (c_tile * nwin) / a.run;
+        s_store<LAYOUT, RT>(a, c_tile, split * a.kmax + seg, lane, acc);
+        if (npend == 2) {  // only with several K slices and a run over three or more tiles
+          s_publish<LAYOUT, RT>(a, pend_tile, pend_contrib, npend, lane);
+          npend = 0;
+        }
+        pend_tile[npend] = c_tile;
+        pend_contrib[npend] = contributors;
+        npend++;
+      }
+#pragma unroll
+      for (int rt = 0; rt < RT; rt++) acc[rt][0] = acc[rt][1] = 0.f;
+      if (c_w == nwin) {
+        c_w = 0;
+        c_tile++;
+      }
+    }
+  }
+  if (npend) s_publish<LAYOUT, RT>(a, pend_tile, pend_contrib, npend, lane);
+  // After a timeout, let the boxes still in flight land (again bounded in time) before the CTA's
+  // shared memory is released.
+  if (st < total) {
+    const int issued = min(total, st + STAGES);
+    const uint64_t t0 = sm100::globaltimer_ns();
+    for (int k = st; k < issued; k++)
+      while (!sm100::mbar_try_wait(full + (k % STAGES), (k / STAGES) & 1) &&
+             sm100::globaltimer_ns() - t0 < kRegWaitLimitNs) {
+      }
+  }
+}
+
 // ---- host side ------------------------------------------------------------------------------------
 int nt_for(int64_t batch) {
   const int nt = (int)((batch + 3) / 4);
@@ -599,20 +1084,116 @@ cudaError_t launch_t(const Args& a, int gx_hint, cudaStream_t st) {
 
 template <int LAYOUT>
 cudaError_t dispatch(const Args& a, int gx_hint, cudaStream_t st) {
+  // the register-decode kernel takes Q2_0_g128 batches 1-4 and base-3 batches 1-2
   switch (bs_for(a.batch)) {
-    case 1: return launch_t<LAYOUT, 1, 2, 1>(a, gx_hint, st);
-    case 2: return launch_t<LAYOUT, 1, 2, 2>(a, gx_hint, st);
-    case 4: return launch_t<LAYOUT, 1, 2, 4>(a, gx_hint, st);
+    case 4:
+      if (LAYOUT == TERN_T3_5PB_G128) return launch_t<LAYOUT, 1, 2, 4>(a, gx_hint, st);
+      break;
     case 8: return launch_t<LAYOUT, 2, 1, 8>(a, gx_hint, st);
     case 16: return launch_t<LAYOUT, 4, 1, 16>(a, gx_hint, st);
     case 32: return launch_t<LAYOUT, 8, 1, 32>(a, gx_hint, st);
-    default: return launch_t<LAYOUT, 16, 1, 64>(a, gx_hint, st);
+    case 64: return launch_t<LAYOUT, 16, 1, 64>(a, gx_hint, st);
+    default: break;
   }
+  return cudaErrorInvalidValue;
+}
+
+template <int LAYOUT, int RT, int BS, int STAGES>
+cudaError_t launch_reg(const CUtensorMap& tc, const CUtensorMap& ts, const Args& a, int grid_x, cudaStream_t st) {
+  const size_t smem = s_smem_bytes(LAYOUT, RT, STAGES, a.gps, BS);
+  auto kern = gemv_reg_kernel<LAYOUT, RT, BS, STAGES>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(grid_x, a.splits), kSThreads, smem, st>>>(tc, ts, a);
+  return cudaGetLastError();
+}
+
+#ifndef TERN_REG_RT
+#define TERN_REG_RT 2
+#endif
+#ifndef TERN_REG_STAGES_Q2
+#define TERN_REG_STAGES_Q2 4
+#endif
+#ifndef TERN_REG_STAGES_T3
+#define TERN_REG_STAGES_T3 3
+#endif
+constexpr int kRegRT = TERN_REG_RT;
+constexpr int kRegStagesQ2 = TERN_REG_STAGES_Q2;
+constexpr int kRegStagesT3 = TERN_REG_STAGES_T3;
+
+bool use_reg_kernel(int32_t layout, int64_t n, int64_t k, int64_t batch) {
+  // (tile, window) unit indices are 32-bit
+  const int64_t units = (n + 16 * kRegRT - 1) / (16 * kRegRT) * s_windows(layout, (int)(k / kGroup));
+  if (units >= ((int64_t)1 << 30)) return false;
+  return layout == TERN_Q2_0_G128 ? batch <= 4 : batch <= 2;
+}
+
+cudaError_t dispatch_reg(const tern_matrix& W, const Args& a, int grid_x, cudaStream_t st) {
+  // tensor maps: codes [n][row data bytes] in boxes of 64 B x tile rows; scales [n][groups] in boxes
+  // of 8 (Q2) or 16 (base-3) groups x tile rows
+  const bool q2 = W.layout == TERN_Q2_0_G128;
+  const uint64_t data_bytes = q2 ? (uint64_t)W.k / 4 : (uint64_t)(W.k + 4) / 5;
+  CUtensorMap tc, ts;
+  if (!tmap_2d(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.codes, data_bytes, (uint64_t)W.n, (uint64_t)W.code_row_stride,
+               kWinBytes, 16 * kRegRT, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  if (!tmap_2d(&ts, CU_TENSOR_MAP_DATA_TYPE_UINT16, W.scales, (uint64_t)(W.k / kGroup), (uint64_t)W.n,
+               (uint64_t)W.scale_row_stride * 2, q2 ? 8 : 16, 16 * kRegRT, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  if (q2) {
+    switch (bs_for(a.batch)) {
+      case 1: return launch_reg<TERN_Q2_0_G128, kRegRT, 1, kRegStagesQ2>(tc, ts, a, grid_x, st);
+      case 2: return launch_reg<TERN_Q2_0_G128, kRegRT, 2, kRegStagesQ2>(tc, ts, a, grid_x, st);
+      default: return launch_reg<TERN_Q2_0_G128, kRegRT, 4, kRegStagesQ2>(tc, ts, a, grid_x, st);
+    }
+  }
+  if (a.batch == 1) return launch_reg<TERN_T3_5PB_G128, kRegRT, 1, kRegStagesT3>(tc, ts, a, grid_x, st);
+  return launch_reg<TERN_T3_5PB_G128, kRegRT, 2, kRegStagesT3>(tc, ts, a, grid_x, st);
 }
 
 }  // namespace
 
+// Register kernel: the fewest K slices whose activation fragments leave room for the target number
+// of CTAs per SM, one full wave of CTAs, and the slice's (tile, window) units spread evenly over
+// the warps.
+static GemvPlan reg_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
+  GemvPlan p{};
+  p.reg = true;
+  const int groups = (int)(k / kGroup);
+  const int unit = (layout == TERN_T3_5PB_G128) ? kT3Window : 2;  // K-slice granularity in groups
+  const int units = (groups + unit - 1) / unit;
+  const int stages = layout == TERN_Q2_0_G128 ? kRegStagesQ2 : kRegStagesT3;
+  const int bs = bs_for(batch);
+  // shared memory of one CTA when kRegCtasPerSm of them share an SM (228 KB, 1 KB reserved each)
+  const size_t cap = (size_t)(228 / kRegCtasPerSm - 1) * 1024;
+  int upc = units;
+  while (upc > 1 && s_smem_bytes(layout, kRegRT, stages, upc * unit, bs) > cap) upc = (upc + 1) / 2;
+  const int splits = (units + upc - 1) / upc;
+  const int gps = std::min(groups, upc * unit);
+  const size_t smem = s_smem_bytes(layout, kRegRT, stages, gps, bs);
+  const int per_sm = std::max(1, std::min(kRegCtasPerSm, (int)(227 * 1024 / (smem + 1024))));
+  p.rows_per_cta = 16 * kRegRT;
+  p.row_blocks = (int)((n + p.rows_per_cta - 1) / p.rows_per_cta);
+  p.splits = splits;
+  p.groups_per_split = gps;
+  const int nwin_full = s_windows(layout, gps);
+  const int64_t u_full = (int64_t)p.row_blocks * nwin_full;
+  // runs of `run` units, at most one per warp of a full wave; the longest run sets the time
+  const int64_t warps = (int64_t)std::max(1, (sms * per_sm) / splits) * kSWarps;
+  p.run = (int)std::max<int64_t>(1, (u_full + warps - 1) / warps);
+  const int64_t runs = (u_full + p.run - 1) / p.run;
+  p.grid_x = (int)((runs + kSWarps - 1) / kSWarps);
+  p.kmax = (nwin_full - 1 + p.run - 1) / p.run + 1;  // runs that can touch one tile
+  const bool whole_tiles = splits == 1 && p.run % nwin_full == 0;
+  if (!whole_tiles) {
+    p.ws_partial_bytes = (size_t)splits * p.kmax * batch * n * sizeof(float);
+    p.ws_bytes = (p.ws_partial_bytes + (size_t)p.row_blocks * sizeof(int) + 15) / 16 * 16;
+  }
+  return p;
+}
+
 GemvPlan gemv_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
+  if (use_reg_kernel(layout, n, k, batch)) return reg_plan(layout, n, k, batch, sms);
   GemvPlan p{};
   const int nt = nt_for(batch);
   const int rt = rt_for(nt);
@@ -655,8 +1236,11 @@ cudaError_t launch_gemv(const tern_matrix& W, const uint16_t* x, int batch, uint
   a.splits = plan.splits;
   a.tiles = plan.row_blocks;
   a.unit = 1u;
-  a.ws = plan.splits > 1 ? static_cast<float*>(workspace) : nullptr;
-  a.counters = plan.splits > 1 ? reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + plan.ws_partial_bytes) : nullptr;
+  a.run = plan.run;
+  a.kmax = plan.kmax;
+  a.ws = plan.ws_bytes ? static_cast<float*>(workspace) : nullptr;
+  a.counters = plan.ws_bytes ? reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + plan.ws_partial_bytes) : nullptr;
+  if (plan.reg) return dispatch_reg(W, a, plan.grid_x, st);
   const int gx_hint = (plan.row_blocks + kWarps - 1) / kWarps;
   if (W.layout == TERN_Q2_0_G128) return dispatch<TERN_Q2_0_G128>(a, gx_hint, st);
   return dispatch<TERN_T3_5PB_G128>(a, gx_hint, st);

@@ -1,9 +1,11 @@
 // Internal declarations shared by the library's translation units (not part of the C ABI).
 #pragma once
 
+#include <cuda.h>
+#include <cuda_runtime.h>
+
 #include <cstddef>
 #include <cstdint>
-#include <cuda_runtime.h>
 
 #include "tern.h"
 
@@ -17,6 +19,11 @@ int64_t row_bytes(int32_t layout, int64_t k);
 // Number of streaming multiprocessors of the current device (cached per device).
 int sm_count();
 
+// 2-D TMA tensor map over [outer][inner] elements with rows row_stride_bytes apart, boxes of
+// box_outer x box_inner, out-of-range elements read as zero; encoded once per distinct argument set.
+bool tmap_2d(CUtensorMap* out, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+             uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw);
+
 // ---- launchers (arguments already validated by the C ABI layer) ----------------------------
 cudaError_t launch_pack(int32_t layout, int64_t n, int64_t k, const uint16_t* w, int64_t w_stride,
                         const uint16_t* s, int64_t s_stride, uint8_t* codes, int64_t c_stride,
@@ -27,11 +34,15 @@ cudaError_t launch_unpack(const tern_matrix& W, uint16_t* w_out, int64_t w_strid
 
 // Split-K plan of the decode GEMV for one (layout, n, k, batch) on a device with `sms` SMs.
 struct GemvPlan {
-  int rows_per_cta;     // output rows one CTA produces
+  bool reg;             // small-batch kernel with in-register decode (else the shared-memory one)
+  int rows_per_cta;     // output rows of one warp tile
   int row_blocks;       // ceil(n / rows_per_cta)
   int splits;           // K slices (1 = no workspace)
   int groups_per_split; // 128-weight groups per slice (a multiple of 5 for base-3 when splits > 1)
-  size_t ws_partial_bytes;  // fp32 partial sums [splits][batch][n]
+  int grid_x;           // register kernel: CTAs per K slice
+  int run;              // register kernel: (tile, window) units per warp run
+  int kmax;             // register kernel: partial-sum slots per tile and K slice
+  size_t ws_partial_bytes;  // fp32 partial sums [splits * slots][batch][n]
   size_t ws_bytes;          // partials + one int32 counter per row block, rounded to 16
 };
 GemvPlan gemv_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms);

@@ -108,10 +108,14 @@ def test_gemv_workspace_size_and_rejection(lib):
                          ctypes.c_void_p(FAKE), need - 16, None) == 4
     assert lib.tern_gemv(ctypes.byref(m), ctypes.c_void_p(FAKE), 1, ctypes.c_void_p(FAKE),
                          ctypes.c_void_p(FAKE + 8), need, None) == 3
-    # a tall matrix needs none
+    # a matrix of one 128-weight group per row is never split and needs none
+    one = _mat(n=4096, k=128, code_row_stride=32, scale_row_stride=8)
+    assert lib.tern_gemv_workspace_bytes(ctypes.byref(one), 1) == 0
+    # the size is a pure function of the arguments; batch outside 1..64 gives 0
     big = _mat(n=151936, k=4096, code_row_stride=1024, scale_row_stride=32)
-    assert lib.tern_gemv_workspace_bytes(ctypes.byref(big), 1) == 0
+    assert lib.tern_gemv_workspace_bytes(ctypes.byref(big), 1) == lib.tern_gemv_workspace_bytes(ctypes.byref(big), 1)
     assert lib.tern_gemv_workspace_bytes(ctypes.byref(big), 0) == 0
+    assert lib.tern_gemv_workspace_bytes(ctypes.byref(big), 65) == 0
     assert lib.tern_gemv_workspace_bytes(None, 1) == 0
 
 
