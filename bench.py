@@ -47,7 +47,7 @@ def _env_int(name, default):
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--steps", type=int, default=12000)
     p.add_argument("--warmup", type=int, default=50)
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--no-extras", action="store_true", help="skip the per-row measurements of the other kernels")
@@ -97,7 +97,8 @@ def profiled_traffic(kernel_key: str):
 
 
 class ClockSampler:
-    """Samples nvidia-smi SM clock / throttle reasons every 200 ms while active."""
+    """Samples nvidia-smi SM clock / throttle reasons every 200 ms; only the samples taken between
+    begin() and end() (the timed region) enter the summary."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -105,9 +106,10 @@ class ClockSampler:
 
     def __init__(self, index: int):
         self.index = index
-        self.rows = []
+        self.rows = []  # (host time, fields)
         self.proc = None
         self.thread = None
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
@@ -116,6 +118,9 @@ class ClockSampler:
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            deadline = time.time() + 5.0  # nvidia-smi takes a moment to print its first sample
+            while not self.rows and time.time() < deadline and self.proc.poll() is None:
+                time.sleep(0.02)
         except Exception:
             self.proc = None
         return self
@@ -124,7 +129,13 @@ class ClockSampler:
         for line in self.proc.stdout:
             parts = [x.strip() for x in line.split(",")]
             if len(parts) >= 9:
-                self.rows.append(parts)
+                self.rows.append((time.time(), parts))
+
+    def begin(self):
+        self.t0 = time.time()
+
+    def end(self):
+        self.t1 = time.time()
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -137,14 +148,17 @@ class ClockSampler:
             self.thread.join(timeout=2)
 
     def summary(self):
-        if not self.rows:
+        rows = [r for (t, r) in self.rows
+                if self.t0 is not None and self.t1 is not None and self.t0 <= t <= self.t1]
+        if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[5 + i].lower() == "active"})
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(self.rows)}
+                "reasons": reasons, "samples": len(rows), "power_w_median": statistics.median(pw) if pw else None}
 
 
 # ----------------------------------------------------------------------------- the native arm
@@ -217,12 +231,14 @@ def run_native(args, rank, world, local_rank):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clk:
+        clk.begin()
         with torch.cuda.stream(stream):
             e0.record(stream)
             for i in range(args.steps):
                 graphs[i % copies].replay()
             e1.record(stream)
         e1.synchronize()
+        clk.end()
     barrier()
     ms = e0.elapsed_time(e1)
     ms = max_over_ranks(torch, ms, world, dev)

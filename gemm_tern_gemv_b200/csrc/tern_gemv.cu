@@ -587,10 +587,10 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(Args a) {
 // The MMA columns are (batch, group-within-window) pairs: a base-3 window touches three groups, so a
 // lane's four k-slots may belong to two groups and the activation fragments are stored per column.
 #ifndef TERN_REG_WARPS
-#define TERN_REG_WARPS 8
+#define TERN_REG_WARPS 16
 #endif
 #ifndef TERN_REG_CTAS_PER_SM
-#define TERN_REG_CTAS_PER_SM 2
+#define TERN_REG_CTAS_PER_SM 1
 #endif
 constexpr int kSWarps = TERN_REG_WARPS;
 constexpr int kSThreads = kSWarps * 32;
@@ -720,9 +720,9 @@ __device__ void s_build_frag(const Args& a, int g0, int ngroups, int nwin_alloc,
 }
 
 // Stream-K bookkeeping of the small-batch kernel. In every K slice the units (tile, window), tile-
-// major, are cut into runs of a.run consecutive units, run i going to warp i of the slice (the last
-// run may be shorter; warps past the last run idle). The runs that touch a tile are consecutive and
-// each writes one partial-sum slot.
+// major, are cut into runs of a.run consecutive units, run i going to warp i / gridDim.x of CTA
+// i % gridDim.x (the last run may be shorter; warps past the last run idle). The runs that touch a
+// tile are consecutive and each writes one partial-sum slot.
 template <int LAYOUT>
 __device__ __forceinline__ int s_nseg(const Args& a, int split, int tile) {  // runs touching a tile in a slice
   const int ng = min(a.gps, a.groups - split * a.gps);
@@ -865,8 +865,9 @@ __global__ void __launch_bounds__(kSThreads, kRegCtasPerSm)
   if (threadIdx.x == 0) *abort_flag = 0;
   __syncwarp();
 
-  // this warp's run of (tile, window) units in the slice (empty past the last run)
-  const int wi = blockIdx.x * kSWarps + warp;
+  // this warp's run of (tile, window) units in the slice (empty past the last run); runs are dealt
+  // to CTAs round-robin so both CTAs on an SM, and all SMs, get the same number of runs (+-1)
+  const int wi = blockIdx.x + warp * gridDim.x;
   const int units = a.tiles * nwin;
   const int u_begin = min(wi * a.run, units);
   const int u_end = min(u_begin + a.run, units);
@@ -926,16 +927,74 @@ __global__ void __launch_bounds__(kSThreads, kRegCtasPerSm)
   for (; st < total; st++) {
     if (!sm100::mbar_wait_bounded(full + c_slot, (st / STAGES) & 1, abort_flag, nullptr, 0u, kRegWaitLimitNs)) break;
     const uint32_t stage_u = ring_u + c_slot * STAGE;
-    // activation fragments of the window
-    uint4 bfr[L::J / 2];
+    // codes of the window; activation fragments follow one code word ahead of the MMAs that use them
+    // (fewer live registers than a whole window's worth, latency still covered)
     const uint32_t fa = fbase + (uint32_t)c_w * fstep;
-#pragma unroll
-    for (int jp = 0; jp < L::J / 2; jp++) bfr[jp] = lds128(fa + jp * kJP);
     uint4 cw[RT][2];
 #pragma unroll
     for (int rt = 0; rt < RT; rt++)
 #pragma unroll
       for (int hr = 0; hr < 2; hr++) cw[rt][hr] = lds128(stage_u + lane_code + (rt * 16 + 8 * hr) * kWinBytes);
+    // fragment pairs a word needs: Q2 word w uses pairs 2w, 2w + 1; base-3 word w uses pairs
+    // floor(5w / 2) .. floor((5w + 4) / 2)
+    constexpr int NB = LAYOUT == TERN_Q2_0_G128 ? 2 : 3;
+    auto pair0 = [](int word) { return LAYOUT == TERN_Q2_0_G128 ? 2 * word : (5 * word) >> 1; };
+    uint4 bcur[NB], bnext[NB];
+#pragma unroll
+    for (int i = 0; i < NB; i++) bcur[i] = lds128(fa + (pair0(0) + i) * kJP);
+    float d[RT][4];
+#pragma unroll
+    for (int word = 0; word < 4; word++) {
+      if (word < 3) {
+#pragma unroll
+        for (int i = 0; i < NB; i++) bnext[i] = lds128(fa + (pair0(word + 1) + i) * kJP);
+      }
+      if (LAYOUT == TERN_Q2_0_G128) {
+        uint32_t wl[RT], wh[RT];
+#pragma unroll
+        for (int rt = 0; rt < RT; rt++) {
+          wl[rt] = word == 0 ? cw[rt][0].x : word == 1 ? cw[rt][0].y : word == 2 ? cw[rt][0].z : cw[rt][0].w;
+          wh[rt] = word == 0 ? cw[rt][1].x : word == 1 ? cw[rt][1].y : word == 2 ? cw[rt][1].z : cw[rt][1].w;
+        }
+#pragma unroll
+        for (int sp = 0; sp < 4; sp++) {
+          const int j = 4 * word + sp;
+          const uint4 bq = bcur[(j >> 1) - pair0(word)];
+          const uint32_t b0 = (j & 1) ? bq.z : bq.x, b1 = (j & 1) ? bq.w : bq.y;
+#pragma unroll
+          for (int rt = 0; rt < RT; rt++) {
+            const uint32_t a0 = slot(wl[rt], mul[2 * sp]), a2 = slot(wl[rt], mul[2 * sp + 1]);
+            const uint32_t a1 = slot(wh[rt], mul[2 * sp]), a3 = slot(wh[rt], mul[2 * sp + 1]);
+            if (j == 0) mma_f16_first(d[rt], a0, a1, a2, a3, b0, b1);
+            else mma_f16(d[rt], a0, a1, a2, a3, b0, b1);
+          }
+        }
+      } else {
+        uint32_t o[RT][2][10];
+#pragma unroll
+        for (int rt = 0; rt < RT; rt++)
+#pragma unroll
+          for (int hr = 0; hr < 2; hr++) {
+            const uint32_t wv = word == 0 ? cw[rt][hr].x : word == 1 ? cw[rt][hr].y : word == 2 ? cw[rt][hr].z : cw[rt][hr].w;
+            dec_t3_word(wv, k0, o[rt][hr]);
+          }
+#pragma unroll
+        for (int m = 0; m < 5; m++) {
+          const int j = 5 * word + m;
+          const uint4 bq = bcur[(j >> 1) - pair0(word)];
+          const uint32_t b0 = (j & 1) ? bq.z : bq.x, b1 = (j & 1) ? bq.w : bq.y;
+#pragma unroll
+          for (int rt = 0; rt < RT; rt++) {
+            if (j == 0) mma_f16_first(d[rt], o[rt][0][2 * m], o[rt][1][2 * m], o[rt][0][2 * m + 1], o[rt][1][2 * m + 1], b0, b1);
+            else mma_f16(d[rt], o[rt][0][2 * m], o[rt][1][2 * m], o[rt][0][2 * m + 1], o[rt][1][2 * m + 1], b0, b1);
+          }
+        }
+      }
+      if (word < 3) {
+#pragma unroll
+        for (int i = 0; i < NB; i++) bcur[i] = bnext[i];
+      }
+    }
     // the two scales this lane's columns use, per row (columns without data have D = 0)
     float sa[RT][2], sb[RT][2];
     {
@@ -957,54 +1016,6 @@ __global__ void __launch_bounds__(kSThreads, kRegCtasPerSm)
             sb[rt][hr] = __half2float(__ushort_as_half((unsigned short)lds16(ra + 2)));
           }
         }
-    }
-    float d[RT][4];
-    if (LAYOUT == TERN_Q2_0_G128) {
-#pragma unroll
-      for (int word = 0; word < 4; word++) {
-        uint32_t wl[RT], wh[RT];
-#pragma unroll
-        for (int rt = 0; rt < RT; rt++) {
-          wl[rt] = word == 0 ? cw[rt][0].x : word == 1 ? cw[rt][0].y : word == 2 ? cw[rt][0].z : cw[rt][0].w;
-          wh[rt] = word == 0 ? cw[rt][1].x : word == 1 ? cw[rt][1].y : word == 2 ? cw[rt][1].z : cw[rt][1].w;
-        }
-#pragma unroll
-        for (int sp = 0; sp < 4; sp++) {
-          const int j = 4 * word + sp;
-          const uint4 bq = bfr[j >> 1];
-          const uint32_t b0 = (j & 1) ? bq.z : bq.x, b1 = (j & 1) ? bq.w : bq.y;
-#pragma unroll
-          for (int rt = 0; rt < RT; rt++) {
-            const uint32_t a0 = slot(wl[rt], mul[2 * sp]), a2 = slot(wl[rt], mul[2 * sp + 1]);
-            const uint32_t a1 = slot(wh[rt], mul[2 * sp]), a3 = slot(wh[rt], mul[2 * sp + 1]);
-            if (j == 0) mma_f16_first(d[rt], a0, a1, a2, a3, b0, b1);
-            else mma_f16(d[rt], a0, a1, a2, a3, b0, b1);
-          }
-        }
-      }
-    } else {
-#pragma unroll
-      for (int word = 0; word < 4; word++) {
-        uint32_t o[RT][2][10];
-#pragma unroll
-        for (int rt = 0; rt < RT; rt++)
-#pragma unroll
-          for (int hr = 0; hr < 2; hr++) {
-            const uint32_t wv = word == 0 ? cw[rt][hr].x : word == 1 ? cw[rt][hr].y : word == 2 ? cw[rt][hr].z : cw[rt][hr].w;
-            dec_t3_word(wv, k0, o[rt][hr]);
-          }
-#pragma unroll
-        for (int m = 0; m < 5; m++) {
-          const int j = 5 * word + m;
-          const uint4 bq = bfr[j >> 1];
-          const uint32_t b0 = (j & 1) ? bq.z : bq.x, b1 = (j & 1) ? bq.w : bq.y;
-#pragma unroll
-          for (int rt = 0; rt < RT; rt++) {
-            if (j == 0) mma_f16_first(d[rt], o[rt][0][2 * m], o[rt][1][2 * m], o[rt][0][2 * m + 1], o[rt][1][2 * m + 1], b0, b1);
-            else mma_f16(d[rt], o[rt][0][2 * m], o[rt][1][2 * m], o[rt][0][2 * m + 1], o[rt][1][2 * m + 1], b0, b1);
-          }
-        }
-      }
     }
     // lane (g, q) holds columns 2q, 2q + 1 of rows g (d[0..1]) and g + 8 (d[2..3]); D = 2 sum t x
 #pragma unroll
@@ -1182,7 +1193,8 @@ static GemvPlan reg_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, in
   const int64_t warps = (int64_t)std::max(1, (sms * per_sm) / splits) * kSWarps;
   p.run = (int)std::max<int64_t>(1, (u_full + warps - 1) / warps);
   const int64_t runs = (u_full + p.run - 1) / p.run;
-  p.grid_x = (int)((runs + kSWarps - 1) / kSWarps);
+  // a full wave of CTAs whenever there are runs for it (runs are dealt round-robin over CTAs)
+  p.grid_x = (int)std::min<int64_t>(std::max(1, (sms * per_sm) / splits), runs);
   p.kmax = (nwin_full - 1 + p.run - 1) / p.run + 1;  // runs that can touch one tile
   const bool whole_tiles = splits == 1 && p.run % nwin_full == 0;
   if (!whole_tiles) {
@@ -1192,7 +1204,18 @@ static GemvPlan reg_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, in
   return p;
 }
 
+// Q2_0_g128 batches from this size on run on the tcgen05 prefill GEMM kernel: its tensor core takes
+// the decoded weights at a fixed rate whatever the number of tokens sharing them, which beats the
+// mma.sync kernels once a weight serves this many rows of x.
+constexpr int kGemmMinBatch = 16;
+
 GemvPlan gemv_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
+  if (layout == TERN_Q2_0_G128 && batch >= kGemmMinBatch && n % 8 == 0) {
+    GemvPlan p{};
+    p.gemm = true;
+    p.splits = 1;
+    return p;
+  }
   if (use_reg_kernel(layout, n, k, batch)) return reg_plan(layout, n, k, batch, sms);
   GemvPlan p{};
   const int nt = nt_for(batch);
@@ -1221,6 +1244,7 @@ GemvPlan gemv_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms)
 
 cudaError_t launch_gemv(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y, void* workspace,
                         const GemvPlan& plan, cudaStream_t st) {
+  if (plan.gemm) return launch_gemm(W, x, batch, y, nullptr, st);
   Args a;
   a.codes = static_cast<const uint8_t*>(W.codes);
   a.cstride = W.code_row_stride;

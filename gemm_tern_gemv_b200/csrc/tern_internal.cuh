@@ -34,6 +34,7 @@ cudaError_t launch_unpack(const tern_matrix& W, uint16_t* w_out, int64_t w_strid
 
 // Split-K plan of the decode GEMV for one (layout, n, k, batch) on a device with `sms` SMs.
 struct GemvPlan {
+  bool gemm;            // Q2_0_g128 with many rows of x: the tcgen05 GEMM kernel (no workspace)
   bool reg;             // small-batch kernel with in-register decode (else the shared-memory one)
   int rows_per_cta;     // output rows of one warp tile
   int row_blocks;       // ceil(n / rows_per_cta)

@@ -140,7 +140,9 @@ TERN_API tern_status tern_unpack(const tern_matrix* W, uint16_t* w_out, int64_t 
 TERN_API size_t tern_gemv_workspace_bytes(const tern_matrix* W, int64_t batch);
 
 /* y[b][n] = sum_g s[n][g] * sum_{k in group g} t[n][k] * x[b][k] for b < batch; fp32
- * accumulation, fp16 result.
+ * accumulation, fp16 result. Small batches run on mma.sync kernels that decode the codes in
+ * registers; Q2_0_g128 batches of 16 or more with n % 8 == 0 run on the tcgen05 kernel of tern_gemm
+ * (no workspace). The result of a call depends only on (W, x, batch) and the device.
  *   x          device fp16 [batch][k], contiguous
  *   y          device fp16 [batch][n], contiguous
  *   workspace  device, >= tern_gemv_workspace_bytes(W, batch) bytes, 16-byte aligned; may be
