@@ -134,7 +134,6 @@ tern_status tern_gemm(const tern_matrix* W, const uint16_t* X, int64_t m, uint16
                       uint32_t* device_status, void* stream) {
   tern_status s = check_matrix(W);
   if (s != TERN_OK) return s;
-  if (W->layout != TERN_Q2_0_G128) return TERN_ERR_UNSUPPORTED;
   if (m <= 0 || m > (int64_t)INT32_MAX || !X || !Y) return TERN_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(Y)) return TERN_ERR_ALIGNMENT;
   if (W->n % 8) return TERN_ERR_ALIGNMENT;  // Y rows are stored as 16-byte vectors

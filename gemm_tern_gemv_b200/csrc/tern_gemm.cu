@@ -40,11 +40,15 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
 
 constexpr int X_STAGE_BYTES = BN * BK * 2;      // 32 KB
 constexpr int A_STAGE_BYTES = BM * BK * 2;      // 16 KB
-constexpr int P_STAGE_BYTES = BM * (BK / 4);    // 2 KB of packed codes
+// Packed codes of a K block, per row: Q2_0_g128 16 bytes; base-3 a 32-byte box at the 16-byte
+// boundary below the block's first byte (the block's 64 trits span at most 14 bytes).
+template <int LAYOUT> constexpr int p_row_bytes() { return LAYOUT == TERN_Q2_0_G128 ? BK / 4 : 32; }
+constexpr int P_STAGE_BYTES = BM * 32;          // room for either layout
 constexpr int OFF_X = 0;
 constexpr int OFF_A = OFF_X + STAGES * X_STAGE_BYTES;
 constexpr int OFF_P = OFF_A + DSTAGES * A_STAGE_BYTES;
-constexpr int OFF_BAR = OFF_P + STAGES * P_STAGE_BYTES;
+constexpr int OFF_LUT = OFF_P + STAGES * P_STAGE_BYTES;  // base-3 byte -> five 2-bit fields
+constexpr int OFF_BAR = OFF_LUT + 256 * 4;
 constexpr int NUM_BARS = 2 * STAGES + 2 * DSTAGES + 4 + 1;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1024
@@ -69,6 +73,39 @@ __device__ __forceinline__ uint32_t pair_2t(uint32_t w, int j) {
   return (x * ((1u << a) + (1u << (a + 14)))) & 0xC000C000u;
 }
 
+// Base-3 K block whose first trit is digit R0 of its first byte: the 64 weights -> fp16 2 s t in the
+// 128-byte-swizzled K-major row `arow`. F[j] holds the five 2-bit two's-complement fields of byte j
+// (table lookup); a pair of weights in one byte is one masked multiply as in pair_2t, a pair across
+// a byte boundary (digit 4, digit 0) is assembled from both bytes. All offsets are compile-time.
+template <int R0>
+__device__ __forceinline__ void t3_block(const uint8_t* prow, const uint32_t* lut, __half2 s2, uint8_t* arow, int rsw) {
+  constexpr int NB = (R0 + 63) / 5 + 1;
+  uint32_t F[NB];
+#pragma unroll
+  for (int j = 0; j < NB; j++) F[j] = lut[prow[j]];
+#pragma unroll
+  for (int c = 0; c < 8; c++) {  // 16-byte chunk c holds k = 8c .. 8c + 7 of the block
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      const int i1 = R0 + 8 * c + 2 * e, i2 = i1 + 1;
+      const int b1 = i1 / 5, d1 = i1 % 5, b2 = i2 / 5;
+      uint32_t two_t;
+      if (b1 == b2) {
+        const uint32_t x = F[b1] & (0xFu << (2 * d1));
+        const uint32_t a = 14 - 2 * d1;
+        two_t = (x * ((1u << a) + (1u << (a + 14)))) & 0xC000C000u;
+      } else {  // digit 4 of byte b1, digit 0 of byte b2
+        two_t = ((F[b1] << 6) & 0x0000C000u) | (F[b2] << 30);
+      }
+      const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&two_t), s2);  // 2 s t, exact
+      o[e] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+    *reinterpret_cast<uint4*>(arow + ((c ^ rsw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+template <int LAYOUT>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w, Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -97,6 +134,17 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) { prefetch_tmap(&tmap_x); prefetch_tmap(&tmap_w); }
+  if (LAYOUT == TERN_T3_5PB_G128) {
+    uint32_t* lut = reinterpret_cast<uint32_t*>(smem + OFF_LUT);
+    for (int v = threadIdx.x; v < 256; v += kThreads) {
+      uint32_t f = 0, r = (uint32_t)v;
+      if (v < 243) {
+#pragma unroll
+        for (int d = 0; d < 5; d++) { f |= (((r % 3u) + 3u) & 3u) << (2 * d); r /= 3u; }  // c - 1 as 2 bits
+      }
+      lut[v] = f;  // an invalid byte reads as five t = 0
+    }
+  }
   if (warp == 1) {
     tmem_alloc(tmem_holder, kTmemCols);
     tmem_relinquish();
@@ -122,9 +170,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(full + s, X_STAGE_BYTES + P_STAGE_BYTES);
+          mbar_arrive_expect_tx(full + s, X_STAGE_BYTES + BM * p_row_bytes<LAYOUT>());
           tma_load_2d(smem + OFF_X + s * X_STAGE_BYTES, &tmap_x, full + s, kb * BK, m0);
-          tma_load_2d(smem + OFF_P + s * P_STAGE_BYTES, &tmap_w, full + s, kb * (BK / 4), n0);
+          const int px = LAYOUT == TERN_Q2_0_G128 ? kb * (BK / 4) : ((kb * BK) / 5) & ~15;
+          tma_load_2d(smem + OFF_P + s * P_STAGE_BYTES, &tmap_w, full + s, px, n0);
           pending[s] = true;
           pend_par[s] = ph;
         }
@@ -223,21 +272,35 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
           ok = false;
           break;
         }
-        const uint4 pk = *reinterpret_cast<const uint4*>(smem + OFF_P + s * P_STAGE_BYTES + r * 16);
         const __half2 s2 = __halves2half2(__ushort_as_half(sbits), __ushort_as_half(sbits));
-        const uint32_t wv[4] = {pk.x, pk.y, pk.z, pk.w};
         uint8_t* arow = smem + OFF_A + d * A_STAGE_BYTES + (r >> 3) * 1024 + (r & 7) * 128;
+        if (LAYOUT == TERN_Q2_0_G128) {
+          const uint4 pk = *reinterpret_cast<const uint4*>(smem + OFF_P + s * P_STAGE_BYTES + r * 16);
+          const uint32_t wv[4] = {pk.x, pk.y, pk.z, pk.w};
 #pragma unroll
-        for (int c = 0; c < 8; c++) {  // 16-byte chunk c holds k = 8c .. 8c + 7
-          const uint32_t w = wv[c >> 1];
-          uint32_t o[4];
+          for (int c = 0; c < 8; c++) {  // 16-byte chunk c holds k = 8c .. 8c + 7
+            const uint32_t w = wv[c >> 1];
+            uint32_t o[4];
 #pragma unroll
-          for (int e = 0; e < 4; e++) {
-            const uint32_t two_t = pair_2t(w, (c & 1) * 4 + e);
-            const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&two_t), s2);  // 2 s t, exact
-            o[e] = *reinterpret_cast<const uint32_t*>(&v);
+            for (int e = 0; e < 4; e++) {
+              const uint32_t two_t = pair_2t(w, (c & 1) * 4 + e);
+              const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&two_t), s2);  // 2 s t, exact
+              o[e] = *reinterpret_cast<const uint32_t*>(&v);
+            }
+            *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
           }
-          *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        } else {
+          // the block's trits start at digit r0 of byte b0; the box starts at the 16-byte boundary below b0
+          const int b0 = (kb * BK) / 5, r0 = (kb * BK) % 5;
+          const uint8_t* prow = smem + OFF_P + s * P_STAGE_BYTES + r * 32 + (b0 & 15);
+          const uint32_t* lut = reinterpret_cast<const uint32_t*>(smem + OFF_LUT);
+          switch (r0) {
+            case 0: t3_block<0>(prow, lut, s2, arow, r & 7); break;
+            case 1: t3_block<1>(prow, lut, s2, arow, r & 7); break;
+            case 2: t3_block<2>(prow, lut, s2, arow, r & 7); break;
+            case 3: t3_block<3>(prow, lut, s2, arow, r & 7); break;
+            default: t3_block<4>(prow, lut, s2, arow, r & 7); break;
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -260,10 +323,12 @@ cudaError_t launch_gemm(const tern_matrix& W, const uint16_t* X, int64_t m, uint
                         cudaStream_t st) {
   CUtensorMap mx, mw;
   const uint64_t k = (uint64_t)W.k, n = (uint64_t)W.n;
+  const bool q2 = W.layout == TERN_Q2_0_G128;
   if (!tmap_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, X, k, (uint64_t)m, k * 2, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  if (!tmap_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.codes, k / 4, n, (uint64_t)W.code_row_stride, BK / 4, BM,
-               CU_TENSOR_MAP_SWIZZLE_NONE))
+  // codes [n][row data bytes]: Q2 boxes of 16 bytes, base-3 boxes of 32 bytes (zero-filled past the data)
+  if (!tmap_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.codes, q2 ? k / 4 : (k + 4) / 5, n, (uint64_t)W.code_row_stride,
+               q2 ? BK / 4 : 32, BM, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   Params p;
   p.m = (int)m;
@@ -275,11 +340,12 @@ cudaError_t launch_gemm(const tern_matrix& W, const uint16_t* X, int64_t m, uint
   p.sstride = W.scale_row_stride;
   p.y = Y;
   p.status = device_status;
-  cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  auto kern = q2 ? gemm_kernel<TERN_Q2_0_G128> : gemm_kernel<TERN_T3_5PB_G128>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int tiles = p.n_tiles * p.m_tiles;
   const int grid = tiles < sm_count() ? tiles : sm_count();
-  gemm_kernel<<<grid, kThreads, SMEM_BYTES, st>>>(mx, mw, p);
+  kern<<<grid, kThreads, SMEM_BYTES, st>>>(mx, mw, p);
   return cudaGetLastError();
 }
 

@@ -1204,13 +1204,13 @@ static GemvPlan reg_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, in
   return p;
 }
 
-// Q2_0_g128 batches from this size on run on the tcgen05 prefill GEMM kernel: its tensor core takes
-// the decoded weights at a fixed rate whatever the number of tokens sharing them, which beats the
-// mma.sync kernels once a weight serves this many rows of x.
+// Batches from this size on run on the tcgen05 prefill GEMM kernel: its tensor core takes the decoded
+// weights at a fixed rate whatever the number of tokens sharing them, which beats the mma.sync
+// kernels once a weight serves this many rows of x.
 constexpr int kGemmMinBatch = 16;
 
 GemvPlan gemv_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
-  if (layout == TERN_Q2_0_G128 && batch >= kGemmMinBatch && n % 8 == 0) {
+  if (batch >= kGemmMinBatch && n % 8 == 0) {
     GemvPlan p{};
     p.gemm = true;
     p.splits = 1;

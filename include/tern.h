@@ -141,8 +141,8 @@ TERN_API size_t tern_gemv_workspace_bytes(const tern_matrix* W, int64_t batch);
 
 /* y[b][n] = sum_g s[n][g] * sum_{k in group g} t[n][k] * x[b][k] for b < batch; fp32
  * accumulation, fp16 result. Small batches run on mma.sync kernels that decode the codes in
- * registers; Q2_0_g128 batches of 16 or more with n % 8 == 0 run on the tcgen05 kernel of tern_gemm
- * (no workspace). The result of a call depends only on (W, x, batch) and the device.
+ * registers; batches of 16 or more with n % 8 == 0 run on the tcgen05 kernel of tern_gemm (no
+ * workspace). The result of a call depends only on (W, x, batch) and the device.
  *   x          device fp16 [batch][k], contiguous
  *   y          device fp16 [batch][n], contiguous
  *   workspace  device, >= tern_gemv_workspace_bytes(W, batch) bytes, 16-byte aligned; may be
@@ -173,7 +173,8 @@ TERN_API tern_status tern_gemv(const tern_matrix* W, const uint16_t* x, int64_t 
  *     streams without ordering between them) race and give wrong results. Order them.
  *   - A matrix / batch whose split-K workspace (tern_gemv_workspace_bytes) exceeds
  *     TERN_GEMV_NOALLOC_SCRATCH_BYTES returns TERN_ERR_WORKSPACE before any launch; batch <= 8
- *     fits for all matrices up to N = 151936, K = 17408.
+ *     fits for N <= 151936 at K = 4096 and for N <= 34816 up to K = 17408, and batches of 16 or
+ *     more with N % 8 == 0 need no scratch.
  * Errors: those of tern_gemv, TERN_ERR_WORKSPACE as above, TERN_ERR_CUDA if the address lookup
  * or the memset fails. */
 TERN_API tern_status tern_gemv_noalloc(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y,
@@ -188,8 +189,10 @@ TERN_API tern_status tern_gemv_noalloc(const tern_matrix* W, const uint16_t* x, 
  *   device_status  device uint32 or NULL: TERN_DEVICE_TIMEOUT is OR-ed in if an internal pipeline
  *                  wait exceeds its bound (the kernel then abandons its work and exits; Y is
  *                  incomplete). The caller zeroes it.
- * Only TERN_Q2_0_G128 is supported (base-3 returns TERN_ERR_UNSUPPORTED).
- * Errors: TERN_ERR_INVALID_ARG, TERN_ERR_UNSUPPORTED, TERN_ERR_ALIGNMENT, TERN_ERR_CUDA. */
+ * Both layouts: a base-3 K block of 64 weights spans at most 14 bytes and is decoded through a
+ * byte -> five-field table; Q2_0_g128 through one masked multiply per pair of weights.
+ * Errors: TERN_ERR_INVALID_ARG, TERN_ERR_UNSUPPORTED (unknown layout), TERN_ERR_ALIGNMENT,
+ * TERN_ERR_CUDA. */
 TERN_API tern_status tern_gemm(const tern_matrix* W, const uint16_t* X, int64_t m, uint16_t* Y,
                       uint32_t* device_status, void* stream);
 

@@ -131,7 +131,8 @@ def test_pack_unpack_gemm_reject(lib):
     assert lib.tern_unpack(ctypes.byref(m), P(FAKE), 1000, None, 0, None, None) == 1
     assert lib.tern_unpack(ctypes.byref(m), P(FAKE), 1028, None, 0, None, None) == 3
     t3 = _mat(layout=2, code_row_stride=208)
-    assert lib.tern_gemm(ctypes.byref(t3), P(FAKE), 16, P(FAKE), None, None) == 2
+    assert lib.tern_gemm(ctypes.byref(t3), P(FAKE), 0, P(FAKE), None, None) == 1  # base-3 accepted up to m
+    assert lib.tern_gemm(ctypes.byref(_mat(layout=3)), P(FAKE), 16, P(FAKE), None, None) == 2
     assert lib.tern_gemm(ctypes.byref(m), P(FAKE), 0, P(FAKE), None, None) == 1
     assert lib.tern_gemm(ctypes.byref(_mat(n=60)), P(FAKE), 16, P(FAKE), None, None) == 3
 

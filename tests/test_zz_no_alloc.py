@@ -46,7 +46,7 @@ def test_noalloc_matches_gemv_twice(layout, n, k, batch):
 
 def test_noalloc_rejects_oversized_scratch():
     # a split-K plan that needs more than the static array is refused before any launch
-    n, k, batch = 151936, 4096, 64
+    n, k, batch = 65536, 17408, 13
     W = T.empty_matrix(T.T3_5PB_G128, n, k)
     need = T.gemv_workspace_bytes(W, batch)
     assert need > 8 * 1024 * 1024
