@@ -353,15 +353,23 @@ def measure_extras(torch, T, dev, peaks, stream):
     ev = lambda: torch.cuda.Event(enable_timing=True)
 
     def timed(fn, reps):
+        # reps back-to-back calls captured in one CUDA graph; device time of a replay / reps (host
+        # launch overhead of the Python binding stays out of the figure)
         with torch.cuda.stream(stream):
             fn()
             torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(reps):
+                    fn()
+            g.replay()
+            torch.cuda.synchronize()
             a, b = ev(), ev()
             a.record(stream)
-            for _ in range(reps):
-                fn()
+            g.replay()
             b.record(stream)
         b.synchronize()
+        del g
         return a.elapsed_time(b) / reps
 
     # ternarize + pack of fp16 latents, 8B shapes (both layouts)
@@ -411,19 +419,32 @@ def measure_extras(torch, T, dev, peaks, stream):
     cache.clear()
     torch.cuda.empty_cache()
 
-    # prefill GEMM M=2048, K=5120, N=17408 (Q2_0_g128) on tcgen05
-    try:
-        M, N, K = 2048, 17408, 5120
-        Wg = make_weights(torch, T, N, K, T.Q2_0_G128, 5, dev)
-        X = torch.randn((M, K), device=dev).to(torch.float16)
-        Y = torch.empty((M, N), dtype=torch.float16, device=dev)
-        ms = timed(lambda: T.gemm(Wg, X, Y=Y), 20)
-        tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
-        res["gemm_q2_2048x17408x5120"] = {"TFLOP/s": round(tf, 1),
-                                          "frac_fp16_peak": round(tf / peaks["bf16_tflops"], 4),
-                                          "peak_TFLOP/s": peaks["bf16_tflops"], "ms": round(ms, 4)}
-    except Exception as e:  # the GEMM is reported, not required for the GEMV metric
-        res["gemm_q2_2048x17408x5120"] = {"error": str(e)[:200]}
+    # activation-side block Hadamard rotation (sign flip + FWHT per 1024-block) in front of a GEMV
+    signs = torch.where(torch.rand(1024, device=dev) < 0.5, -1, 1).to(torch.int8)
+    for b, k in ((1, 4096), (1, 12288), (64, 17408)):
+        xr = torch.randn((b, k), device=dev).to(torch.float16)
+        yr = torch.empty_like(xr)
+        ms = timed(lambda: T.hadamard_rotate(xr, signs, y=yr), 50)
+        nb = 2 * (2 * b * k) + 1024
+        res[f"rotate_b{b}_k{k}"] = {"us": round(ms * 1e3, 2), "GB/s": round(nb / (ms * 1e-3) / 1e9, 1),
+                                    "note": "latency-bound (a few KB per call)" if b == 1 else "HBM"}
+
+    # prefill GEMM M=2048, K=5120, N=17408 on tcgen05, both layouts (the prefill config is Q2_0_g128;
+    # the base-3 line is the same product on the denser layout)
+    M, N, K = 2048, 17408, 5120
+    X = torch.randn((M, K), device=dev).to(torch.float16)
+    Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    for layout, lname in ((T.Q2_0_G128, "q2"), (T.T3_5PB_G128, "t3")):
+        key = f"gemm_{lname}_2048x17408x5120"
+        try:
+            Wg = make_weights(torch, T, N, K, layout, 5, dev)
+            ms = timed(lambda: T.gemm(Wg, X, Y=Y), 20)
+            tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+            res[key] = {"TFLOP/s": round(tf, 1), "frac_fp16_peak": round(tf / peaks["bf16_tflops"], 4),
+                        "peak_TFLOP/s": peaks["bf16_tflops"], "ms": round(ms, 4)}
+            del Wg
+        except Exception as e:  # the GEMM is reported, not required for the GEMV metric
+            res[key] = {"error": str(e)[:200]}
     return res
 
 

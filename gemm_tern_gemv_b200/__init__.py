@@ -57,6 +57,8 @@ SIGNATURES = {
                                          ctypes.c_void_p]),
     "tern_gemm": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                  ctypes.c_void_p, ctypes.c_void_p]),
+    "tern_hadamard_rotate": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                            ctypes.c_void_p, ctypes.c_void_p]),
     "tern_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "tern_version": (ctypes.c_int32, []),
 }
@@ -242,6 +244,21 @@ def gemv_noalloc(W: TernMatrix, x, y=None):
     st = lib().tern_gemv_noalloc(ctypes.byref(c), _ptr(x), x.shape[0], _ptr(y), _stream_handle())
     _check(st, "tern_gemv_noalloc")
     return y
+
+
+def hadamard_rotate(x, signs, y=None):
+    """y = R x per 1024-block of every row, R = H S / 32 (tern_hadamard_rotate); x fp16 [batch][k] or
+    [k], signs int8 [1024] on the device (negative = -1). y may be x itself (in place)."""
+    torch = _torch()
+    squeeze = x.dim() == 1
+    x2 = (x.unsqueeze(0) if squeeze else x).contiguous()
+    if y is None:
+        y = torch.empty_like(x2)
+    elif squeeze:
+        y = y.view(1, -1)
+    st = lib().tern_hadamard_rotate(_ptr(x2), x2.shape[0], x2.shape[1], _ptr(signs), _ptr(y), _stream_handle())
+    _check(st, "tern_hadamard_rotate")
+    return y[0] if squeeze else y
 
 
 def gemm(W: TernMatrix, X, Y=None, status=None):

@@ -141,6 +141,14 @@ tern_status tern_gemm(const tern_matrix* W, const uint16_t* X, int64_t m, uint16
   return from_cuda(launch_gemm(*W, X, m, Y, device_status, static_cast<cudaStream_t>(stream)));
 }
 
+tern_status tern_hadamard_rotate(const uint16_t* x, int64_t batch, int64_t k, const int8_t* signs, uint16_t* y,
+                                 void* stream) {
+  if (!x || !y || !signs || batch < 1 || k <= 0 || k % 1024) return TERN_ERR_INVALID_ARG;
+  if (batch > (int64_t)INT32_MAX / (k / 1024) || batch * k > (int64_t)1 << 40) return TERN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & 1u) return TERN_ERR_ALIGNMENT;
+  return from_cuda(launch_rotate(x, batch, k, signs, y, static_cast<cudaStream_t>(stream)));
+}
+
 const char* tern_status_string(tern_status status) {
   switch (status) {
     case TERN_OK: return "ok";

@@ -1207,7 +1207,7 @@ static GemvPlan reg_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, in
 // Batches from this size on run on the tcgen05 prefill GEMM kernel: its tensor core takes the decoded
 // weights at a fixed rate whatever the number of tokens sharing them, which beats the mma.sync
 // kernels once a weight serves this many rows of x.
-constexpr int kGemmMinBatch = 16;
+constexpr int kGemmMinBatch = 17;
 
 GemvPlan gemv_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
   if (batch >= kGemmMinBatch && n % 8 == 0) {

@@ -57,4 +57,7 @@ tern_status gemv_noalloc(const tern_matrix& W, const uint16_t* x, int batch, uin
 cudaError_t launch_gemm(const tern_matrix& W, const uint16_t* X, int64_t m, uint16_t* Y,
                         uint32_t* device_status, cudaStream_t st);
 
+cudaError_t launch_rotate(const uint16_t* x, int64_t batch, int64_t k, const int8_t* signs, uint16_t* y,
+                          cudaStream_t st);
+
 }  // namespace tern

@@ -141,7 +141,7 @@ TERN_API size_t tern_gemv_workspace_bytes(const tern_matrix* W, int64_t batch);
 
 /* y[b][n] = sum_g s[n][g] * sum_{k in group g} t[n][k] * x[b][k] for b < batch; fp32
  * accumulation, fp16 result. Small batches run on mma.sync kernels that decode the codes in
- * registers; batches of 16 or more with n % 8 == 0 run on the tcgen05 kernel of tern_gemm (no
+ * registers; batches of 17 or more with n % 8 == 0 run on the tcgen05 kernel of tern_gemm (no
  * workspace). The result of a call depends only on (W, x, batch) and the device.
  *   x          device fp16 [batch][k], contiguous
  *   y          device fp16 [batch][n], contiguous
@@ -173,7 +173,7 @@ TERN_API tern_status tern_gemv(const tern_matrix* W, const uint16_t* x, int64_t 
  *     streams without ordering between them) race and give wrong results. Order them.
  *   - A matrix / batch whose split-K workspace (tern_gemv_workspace_bytes) exceeds
  *     TERN_GEMV_NOALLOC_SCRATCH_BYTES returns TERN_ERR_WORKSPACE before any launch; batch <= 8
- *     fits for N <= 151936 at K = 4096 and for N <= 34816 up to K = 17408, and batches of 16 or
+ *     fits for N <= 151936 at K = 4096 and for N <= 34816 up to K = 17408, and batches of 17 or
  *     more with N % 8 == 0 need no scratch.
  * Errors: those of tern_gemv, TERN_ERR_WORKSPACE as above, TERN_ERR_CUDA if the address lookup
  * or the memset fails. */
@@ -195,6 +195,22 @@ TERN_API tern_status tern_gemv_noalloc(const tern_matrix* W, const uint16_t* x, 
  * TERN_ERR_CUDA. */
 TERN_API tern_status tern_gemm(const tern_matrix* W, const uint16_t* X, int64_t m, uint16_t* Y,
                       uint32_t* device_status, void* stream);
+
+/* ---- activation-side block Hadamard rotation ------------------------------------------------ */
+
+/* y = R x for every 1024-element block of every row, R = H S / 32 ("Ternary Bonsai 2 27B ..."
+ * discuss.pytorch.kr, section "블록 단위 하다마드 회전": stored weights live in the basis
+ * R = H_n S / sqrt(n), n = 1024, and a layer computes W (R x); section "처리량": the sign flip and
+ * the block fast Walsh-Hadamard transform precede every projection):
+ *   y[b][1024 j + i] = (1/32) sum_m H[i][m] * sgn(signs[m]) * x[b][1024 j + m],
+ * H the Sylvester-order Walsh-Hadamard matrix, H[i][m] = (-1)^popcount(i & m).
+ *   x, y   device fp16 [batch][k], contiguous, k a positive multiple of 1024; y may equal x
+ *   signs  device int8 [1024], the diagonal of S: negative entries are -1, all others +1
+ * fp32 butterflies, fp16 result rounded once; stream-ordered, no allocation.
+ * Errors: TERN_ERR_INVALID_ARG (NULL pointer, batch < 1, k not a positive multiple of 1024,
+ *         batch * k too large), TERN_ERR_ALIGNMENT (x or y not 2-byte aligned), TERN_ERR_CUDA. */
+TERN_API tern_status tern_hadamard_rotate(const uint16_t* x, int64_t batch, int64_t k, const int8_t* signs,
+                                          uint16_t* y, void* stream);
 
 /* Static description of a status code (never NULL). */
 TERN_API const char* tern_status_string(tern_status status);

@@ -30,7 +30,8 @@ def _declared():
 def test_header_declares_the_boundary():
     names = _declared()
     for n in ("tern_pack", "tern_unpack", "tern_gemv", "tern_gemm", "tern_gemv_workspace_bytes",
-              "tern_row_bytes", "tern_packed_bytes", "tern_bits_per_weight", "tern_status_string"):
+              "tern_row_bytes", "tern_packed_bytes", "tern_bits_per_weight", "tern_status_string",
+              "tern_hadamard_rotate"):
         assert n in names
 
 
@@ -142,3 +143,15 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(T, "LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(RuntimeError, match="missing"):
         T.lib()
+
+
+def test_hadamard_rotate_rejects_before_launch(lib):
+    P = lambda v: ctypes.c_void_p(v)
+    f = lib.tern_hadamard_rotate
+    assert f(None, 1, 1024, P(FAKE), P(FAKE), None) == 1
+    assert f(P(FAKE), 1, 1024, None, P(FAKE), None) == 1
+    assert f(P(FAKE), 0, 1024, P(FAKE), P(FAKE), None) == 1
+    assert f(P(FAKE), 1, 1000, P(FAKE), P(FAKE), None) == 1
+    assert f(P(FAKE), 1, 0, P(FAKE), P(FAKE), None) == 1
+    assert f(P(FAKE + 1), 1, 1024, P(FAKE), P(FAKE), None) == 3
+    assert f(P(FAKE), 1, 1024, P(FAKE), P(FAKE + 1), None) == 3
