@@ -57,6 +57,12 @@ SIGNATURES = {
                                          ctypes.c_void_p]),
     "tern_gemm": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                  ctypes.c_void_p, ctypes.c_void_p]),
+    "tern_pack_flips": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64,
+                                       ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                       ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]),
+    "tern_gemv_t_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(TernMatrixC), ctypes.c_int64]),
+    "tern_gemv_t": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "tern_hadamard_rotate": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
                                             ctypes.c_void_p, ctypes.c_void_p]),
     "tern_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -181,6 +187,24 @@ def pack(w, scales, layout: int = Q2_0_G128, out: TernMatrix | None = None) -> T
     return out
 
 
+def pack_flips(w, scales, prev: TernMatrix, out: TernMatrix | None = None, flips=None):
+    """Re-pack w like pack() and count the weights whose code changed against `prev`
+    (tern_pack_flips). Returns (matrix, flips) with flips a device int64 tensor (added to when given)."""
+    torch = _torch()
+    n, k = w.shape
+    scales = as_scales(scales, k)
+    if out is None:
+        codes = torch.empty((n, row_bytes(prev.layout, k)), dtype=torch.uint8, device=w.device)
+        out = TernMatrix(prev.layout, n, k, codes, scales)
+    if flips is None:
+        flips = torch.zeros(1, dtype=torch.int64, device=w.device)
+    st = lib().tern_pack_flips(prev.layout, n, k, _ptr(w), w.stride(0), _ptr(scales), scales.stride(0),
+                               _ptr(out.codes), out.codes.stride(0), _ptr(prev.codes), prev.codes.stride(0),
+                               _ptr(flips), _stream_handle())
+    _check(st, "tern_pack_flips")
+    return out, flips
+
+
 def from_packed(codes, scales, layout: int, k: int) -> TernMatrix:
     """Wrap already-packed codes (uint8 [n][>=row_bytes]) and scales as a TernMatrix (device copies)."""
     torch = _torch()
@@ -244,6 +268,25 @@ def gemv_noalloc(W: TernMatrix, x, y=None):
     st = lib().tern_gemv_noalloc(ctypes.byref(c), _ptr(x), x.shape[0], _ptr(y), _stream_handle())
     _check(st, "tern_gemv_noalloc")
     return y
+
+
+def gemv_t(W: TernMatrix, dy, dx=None, workspace=None):
+    """dx [batch][k] = dy [batch][n] @ W (tern_gemv_t, the STE-backward input gradient), batch <= 8."""
+    torch = _torch()
+    if dy.dim() == 1:
+        dy = dy.unsqueeze(0)
+    dy = dy.contiguous()
+    batch = dy.shape[0]
+    if dx is None:
+        dx = torch.empty((batch, W.k), dtype=torch.float16, device=dy.device)
+    c = W.c()
+    if workspace is None:
+        nb = int(lib().tern_gemv_t_workspace_bytes(ctypes.byref(c), batch))
+        workspace = torch.empty(nb, dtype=torch.uint8, device=dy.device) if nb else None
+    wsb = workspace.numel() if workspace is not None else 0
+    st = lib().tern_gemv_t(ctypes.byref(c), _ptr(dy), batch, _ptr(dx), _ptr(workspace), wsb, _stream_handle())
+    _check(st, "tern_gemv_t")
+    return dx
 
 
 def hadamard_rotate(x, signs, y=None):

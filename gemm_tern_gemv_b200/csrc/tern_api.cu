@@ -71,9 +71,10 @@ double tern_bits_per_weight(int32_t layout, int64_t k) {
   return (double)(rb * 8 + (k / kGroup) * 16) / (double)k;
 }
 
-tern_status tern_pack(int32_t layout, int64_t n, int64_t k, const uint16_t* w, int64_t w_row_stride,
-                      const uint16_t* scales, int64_t scale_row_stride, void* codes,
-                      int64_t code_row_stride, void* stream) {
+static tern_status pack_common(int32_t layout, int64_t n, int64_t k, const uint16_t* w, int64_t w_row_stride,
+                               const uint16_t* scales, int64_t scale_row_stride, void* codes,
+                               int64_t code_row_stride, const void* prev, int64_t prev_row_stride,
+                               uint64_t* flips, void* stream) {
   if (layout != TERN_Q2_0_G128 && layout != TERN_T3_5PB_G128) return TERN_ERR_UNSUPPORTED;
   if (n <= 0 || k <= 0 || k % kGroup || n > (int64_t)INT32_MAX || k > (int64_t)INT32_MAX / 2)
     return TERN_ERR_INVALID_ARG;
@@ -82,9 +83,30 @@ tern_status tern_pack(int32_t layout, int64_t n, int64_t k, const uint16_t* w, i
     return TERN_ERR_INVALID_ARG;
   if (!aligned16(w) || !aligned16(scales) || !aligned16(codes)) return TERN_ERR_ALIGNMENT;
   if (w_row_stride % 8 || scale_row_stride % 8 || code_row_stride % 16) return TERN_ERR_ALIGNMENT;
+  if (prev) {
+    if (!flips || prev_row_stride < row_bytes(layout, k)) return TERN_ERR_INVALID_ARG;
+    if (!aligned16(prev) || prev_row_stride % 16 || (reinterpret_cast<uintptr_t>(flips) & 7u)) return TERN_ERR_ALIGNMENT;
+  }
   return from_cuda(launch_pack(layout, n, k, w, w_row_stride, scales, scale_row_stride,
                                static_cast<uint8_t*>(codes), code_row_stride,
-                               static_cast<cudaStream_t>(stream)));
+                               static_cast<const uint8_t*>(prev), prev_row_stride,
+                               reinterpret_cast<unsigned long long*>(flips), static_cast<cudaStream_t>(stream)));
+}
+
+tern_status tern_pack(int32_t layout, int64_t n, int64_t k, const uint16_t* w, int64_t w_row_stride,
+                      const uint16_t* scales, int64_t scale_row_stride, void* codes,
+                      int64_t code_row_stride, void* stream) {
+  return pack_common(layout, n, k, w, w_row_stride, scales, scale_row_stride, codes, code_row_stride, nullptr, 0,
+                     nullptr, stream);
+}
+
+tern_status tern_pack_flips(int32_t layout, int64_t n, int64_t k, const uint16_t* w, int64_t w_row_stride,
+                            const uint16_t* scales, int64_t scale_row_stride, void* codes, int64_t code_row_stride,
+                            const void* prev_codes, int64_t prev_row_stride, uint64_t* flips, void* stream) {
+  if (!prev_codes || !flips) return TERN_ERR_INVALID_ARG;
+  if (prev_codes == codes) return TERN_ERR_INVALID_ARG;  // the previous codes must survive the pack
+  return pack_common(layout, n, k, w, w_row_stride, scales, scale_row_stride, codes, code_row_stride, prev_codes,
+                     prev_row_stride, flips, stream);
 }
 
 tern_status tern_unpack(const tern_matrix* W, uint16_t* w_out, int64_t w_row_stride, int8_t* t_out,
@@ -139,6 +161,27 @@ tern_status tern_gemm(const tern_matrix* W, const uint16_t* X, int64_t m, uint16
   if (W->n % 8) return TERN_ERR_ALIGNMENT;  // Y rows are stored as 16-byte vectors
   if (device_status && (reinterpret_cast<uintptr_t>(device_status) & 3u)) return TERN_ERR_ALIGNMENT;
   return from_cuda(launch_gemm(*W, X, m, Y, device_status, static_cast<cudaStream_t>(stream)));
+}
+
+size_t tern_gemv_t_workspace_bytes(const tern_matrix* W, int64_t batch) {
+  if (!W || W->n <= 0 || W->k <= 0 || W->k % kGroup) return 0;
+  if (W->layout != TERN_Q2_0_G128 && W->layout != TERN_T3_5PB_G128) return 0;
+  if (batch < 1 || batch > TERN_GEMV_T_MAX_BATCH) return 0;
+  return gemv_t_plan(W->layout, W->n, W->k, batch, sm_count()).ws_bytes;
+}
+
+tern_status tern_gemv_t(const tern_matrix* W, const uint16_t* dy, int64_t batch, uint16_t* dx, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  tern_status s = check_matrix(W);
+  if (s != TERN_OK) return s;
+  if (batch < 1 || batch > TERN_GEMV_T_MAX_BATCH || !dy || !dx) return TERN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(dy) | reinterpret_cast<uintptr_t>(dx)) & 1u) return TERN_ERR_ALIGNMENT;
+  const GemvTPlan plan = gemv_t_plan(W->layout, W->n, W->k, batch, sm_count());
+  if (plan.ws_bytes) {
+    if (!workspace || workspace_bytes < plan.ws_bytes) return TERN_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return TERN_ERR_ALIGNMENT;
+  }
+  return from_cuda(launch_gemv_t(*W, dy, (int)batch, dx, workspace, plan, static_cast<cudaStream_t>(stream)));
 }
 
 tern_status tern_hadamard_rotate(const uint16_t* x, int64_t batch, int64_t k, const int8_t* signs, uint16_t* y,

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstddef>
 #include <cstdint>
 
@@ -25,9 +26,10 @@ bool tmap_2d(CUtensorMap* out, CUtensorMapDataType dt, const void* base, uint64_
              uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw);
 
 // ---- launchers (arguments already validated by the C ABI layer) ----------------------------
+// prev / flips: optional previous packing of the same matrix and the flip counter it feeds
 cudaError_t launch_pack(int32_t layout, int64_t n, int64_t k, const uint16_t* w, int64_t w_stride,
                         const uint16_t* s, int64_t s_stride, uint8_t* codes, int64_t c_stride,
-                        cudaStream_t st);
+                        const uint8_t* prev, int64_t p_stride, unsigned long long* flips, cudaStream_t st);
 
 cudaError_t launch_unpack(const tern_matrix& W, uint16_t* w_out, int64_t w_stride, int8_t* t_out,
                           int64_t t_stride, int32_t* invalid_count, cudaStream_t st);
@@ -56,6 +58,17 @@ tern_status gemv_noalloc(const tern_matrix& W, const uint16_t* x, int batch, uin
 
 cudaError_t launch_gemm(const tern_matrix& W, const uint16_t* X, int64_t m, uint16_t* Y,
                         uint32_t* device_status, cudaStream_t st);
+
+// Transposed product dx = W^T dy: column blocks x row slices; fp32 partials per slice when sliced.
+struct GemvTPlan {
+  int col_blocks;
+  int slices;
+  int64_t rows_per_slice;
+  size_t ws_bytes;
+};
+GemvTPlan gemv_t_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms);
+cudaError_t launch_gemv_t(const tern_matrix& W, const uint16_t* dy, int batch, uint16_t* dx, void* workspace,
+                          const GemvTPlan& plan, cudaStream_t st);
 
 cudaError_t launch_rotate(const uint16_t* x, int64_t batch, int64_t k, const int8_t* signs, uint16_t* y,
                           cudaStream_t st);

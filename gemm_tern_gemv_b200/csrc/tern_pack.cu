@@ -29,8 +29,11 @@ __device__ __forceinline__ int ternary_value(uint16_t wbits, float s_abs, bool s
 __global__ void __launch_bounds__(kThreads) pack_q2_kernel(const uint16_t* __restrict__ w, int64_t w_stride,
                                                            const uint16_t* __restrict__ s, int64_t s_stride,
                                                            uint8_t* __restrict__ codes, int64_t c_stride,
+                                                           const uint8_t* __restrict__ prev, int64_t p_stride,
+                                                           unsigned long long* __restrict__ flips,
                                                            int64_t n, int chunks_per_row) {
   const int64_t total = n * chunks_per_row;
+  int flipped = 0;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t row = i / chunks_per_row;
     const int ch = (int)(i - row * chunks_per_row);
@@ -57,6 +60,19 @@ __global__ void __launch_bounds__(kThreads) pack_q2_kernel(const uint16_t* __res
       out[word] = acc;
     }
     *reinterpret_cast<uint4*>(codes + row * c_stride + (int64_t)ch * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+    if (prev) {  // a weight flips when its 2-bit field differs from the previous packing
+      const uint4 pv = __ldg(reinterpret_cast<const uint4*>(prev + row * p_stride + (int64_t)ch * 16));
+      const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+      for (int word = 0; word < 4; word++) {
+        const uint32_t d = out[word] ^ pw[word];
+        flipped += __popc((d | (d >> 1)) & 0x55555555u);
+      }
+    }
+  }
+  if (flips) {
+    flipped = __reduce_add_sync(0xFFFFFFFFu, flipped);
+    if ((threadIdx.x & 31) == 0 && flipped) atomicAdd(flips, (unsigned long long)flipped);
   }
 }
 
@@ -64,8 +80,11 @@ __global__ void __launch_bounds__(kThreads) pack_q2_kernel(const uint16_t* __res
 __global__ void __launch_bounds__(kThreads) pack_t3_kernel(const uint16_t* __restrict__ w, int64_t w_stride,
                                                            const uint16_t* __restrict__ s, int64_t s_stride,
                                                            uint8_t* __restrict__ codes, int64_t c_stride,
+                                                           const uint8_t* __restrict__ prev, int64_t p_stride,
+                                                           unsigned long long* __restrict__ flips,
                                                            int64_t n, int k, int chunks_per_row) {
   const int64_t total = n * chunks_per_row;
+  int flipped = 0;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t row = i / chunks_per_row;
     const int ch = (int)(i - row * chunks_per_row);
@@ -103,6 +122,25 @@ __global__ void __launch_bounds__(kThreads) pack_t3_kernel(const uint16_t* __res
       out[word] = acc;
     }
     *reinterpret_cast<uint4*>(codes + row * c_stride + (int64_t)ch * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+    if (prev) {  // a weight (k < K) flips when its base-3 digit differs from the previous packing
+      const uint4 pv = __ldg(reinterpret_cast<const uint4*>(prev + row * p_stride + (int64_t)ch * 16));
+      const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+      for (int b = 0; b < 16; b++) {
+        uint32_t old = (pw[b / 4] >> (8 * (b % 4))) & 0xFFu;
+        const uint32_t neu = (out[b / 4] >> (8 * (b % 4))) & 0xFFu;
+        if (old == neu) continue;
+#pragma unroll
+        for (int f = 0; f < 5; f++) {
+          flipped += (old % 3u != c[5 * b + f]) && (k0 + 5 * b + f < k);
+          old /= 3u;
+        }
+      }
+    }
+  }
+  if (flips) {
+    flipped = __reduce_add_sync(0xFFFFFFFFu, flipped);
+    if ((threadIdx.x & 31) == 0 && flipped) atomicAdd(flips, (unsigned long long)flipped);
   }
 }
 
@@ -194,13 +232,15 @@ int grid_for(int64_t work) {
 
 cudaError_t launch_pack(int32_t layout, int64_t n, int64_t k, const uint16_t* w, int64_t w_stride,
                         const uint16_t* s, int64_t s_stride, uint8_t* codes, int64_t c_stride,
-                        cudaStream_t st) {
+                        const uint8_t* prev, int64_t p_stride, unsigned long long* flips, cudaStream_t st) {
   const int chunks = (int)(row_bytes(layout, k) / 16);
   const int grid = grid_for(n * chunks);
   if (layout == TERN_Q2_0_G128)
-    pack_q2_kernel<<<grid, kThreads, 0, st>>>(w, w_stride, s, s_stride, codes, c_stride, n, chunks);
+    pack_q2_kernel<<<grid, kThreads, 0, st>>>(w, w_stride, s, s_stride, codes, c_stride, prev, p_stride, flips, n,
+                                              chunks);
   else
-    pack_t3_kernel<<<grid, kThreads, 0, st>>>(w, w_stride, s, s_stride, codes, c_stride, n, (int)k, chunks);
+    pack_t3_kernel<<<grid, kThreads, 0, st>>>(w, w_stride, s, s_stride, codes, c_stride, prev, p_stride, flips, n,
+                                              (int)k, chunks);
   return cudaGetLastError();
 }
 

@@ -121,6 +121,23 @@ TERN_API tern_status tern_pack(int32_t layout, int64_t n, int64_t k,
                       const uint16_t* scales, int64_t scale_row_stride,
                       void* codes, int64_t code_row_stride, void* stream);
 
+/* tern_pack that also counts code flips against the previous packing of the same matrix: the QAT
+ * loop watches how many weights change their code from one step to the next ("Metal 환경에서 ...
+ * Bonsai 8B를 파인튜닝", molayo1419.me, paragraph "그것을 파인튜닝하는 방법" and its lr study: flips,
+ * not the loss, show whether training moves the model).
+ *   prev_codes       device uint8 [n][prev_row_stride]: the previous packed codes, same layout and
+ *                    k; must not overlap `codes`
+ *   flips            device uint64: the number of weights (k < K) whose code field (Q2 2-bit field,
+ *                    base-3 digit) differs from prev_codes is ADDED (the caller zeroes it); for
+ *                    valid codes that is the number of weights whose t changed
+ * Errors: those of tern_pack; TERN_ERR_INVALID_ARG for NULL prev_codes / flips, prev_codes ==
+ *         codes or a short prev_row_stride; TERN_ERR_ALIGNMENT for a misaligned prev_codes,
+ *         prev_row_stride or flips. */
+TERN_API tern_status tern_pack_flips(int32_t layout, int64_t n, int64_t k, const uint16_t* w, int64_t w_row_stride,
+                                     const uint16_t* scales, int64_t scale_row_stride, void* codes,
+                                     int64_t code_row_stride, const void* prev_codes, int64_t prev_row_stride,
+                                     uint64_t* flips, void* stream);
+
 /* ---- unpack (test / debug path; the products never call it) ------------------------------ */
 
 /* Expands W to dense form. Either output may be NULL, not both.
@@ -195,6 +212,28 @@ TERN_API tern_status tern_gemv_noalloc(const tern_matrix* W, const uint16_t* x, 
  * TERN_ERR_CUDA. */
 TERN_API tern_status tern_gemm(const tern_matrix* W, const uint16_t* X, int64_t m, uint16_t* Y,
                       uint32_t* device_status, void* stream);
+
+/* ---- transposed product (STE backward) ------------------------------------------------------ */
+
+#define TERN_GEMV_T_MAX_BATCH 8
+
+/* Bytes of fp32 workspace tern_gemv_t needs (0 when it needs none); a function of (layout, n, k,
+ * batch) and the device's SM count. Returns 0 also for invalid arguments. */
+TERN_API size_t tern_gemv_t_workspace_bytes(const tern_matrix* W, int64_t batch);
+
+/* dx[b][k] = sum_n s[n][k/128] * t[n][k] * dy[b][n] for b < batch: the input gradient W^T dy of the
+ * straight-through-estimator backward through a ternary layer ("Metal 환경에서 ... Bonsai 8B를
+ * 파인튜닝", molayo1419.me, paragraph "그것을 파인튜닝하는 방법": the latents are trained through
+ * the ternarized forward). fp32 accumulation, fp16 result; deterministic (row slices are summed
+ * in order).
+ *   dy         device fp16 [batch][n], contiguous;  dx device fp16 [batch][k], contiguous
+ *   workspace  device, >= tern_gemv_t_workspace_bytes(W, batch) bytes, 16-byte aligned; may be NULL
+ *              when that size is 0. Calls that share a workspace must not overlap on the GPU.
+ * Errors: TERN_ERR_INVALID_ARG (batch outside 1..8, NULL pointer, bad matrix), TERN_ERR_UNSUPPORTED,
+ *         TERN_ERR_ALIGNMENT (dy / dx not 2-byte aligned, workspace not 16-byte aligned, matrix
+ *         alignment), TERN_ERR_WORKSPACE, TERN_ERR_CUDA. */
+TERN_API tern_status tern_gemv_t(const tern_matrix* W, const uint16_t* dy, int64_t batch, uint16_t* dx,
+                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---- activation-side block Hadamard rotation ------------------------------------------------ */
 

@@ -159,6 +159,24 @@ def count_invalid(codes: np.ndarray, layout: int, n: int, k: int) -> int:
     return int((codes[:, kk // 5] > 242).sum())
 
 
+def count_flips(old_codes: np.ndarray, new_codes: np.ndarray, layout: int, k: int) -> int:
+    """Weights (row, k < K) whose code field differs between two packings of one matrix: the
+    2-bit field (Q2) or the base-3 digit (T3), read straight from the bytes as the layout defines
+    them (the QAT flip count of [Metal-8B]; for valid codes this is the number of changed t)."""
+    old = np.asarray(old_codes, dtype=np.uint8)
+    new = np.asarray(new_codes, dtype=np.uint8)
+    _check(layout, k)
+    kk = np.arange(k)
+    if layout == Q2_0_G128:
+        f_old = (old[:, kk // 4] >> (2 * (kk % 4))) & 3
+        f_new = (new[:, kk // 4] >> (2 * (kk % 4))) & 3
+    else:
+        p = np.array(_POW3)[kk % 5]
+        f_old = (old[:, kk // 5].astype(np.int64) // p) % 3
+        f_new = (new[:, kk // 5].astype(np.int64) // p) % 3
+    return int((f_old != f_new).sum())
+
+
 def dequantize(t: np.ndarray, scales: np.ndarray) -> np.ndarray:
     """fp64 w[n][k] = s[n][k/128] * t[n][k]  ([velog-27B] "포맷의 정체"; [Bonsai2] eq. w_i)."""
     n, k = t.shape
@@ -201,6 +219,20 @@ def gemv(codes, scales, x, layout: int, k: int, rows=None):
     y = xd @ w.T
     a = np.abs(xd) @ np.abs(w).T
     return y, a
+
+
+def gemv_t(codes, scales, dy, layout: int, k: int, cols=None):
+    """dx_ref[b][k] = sum_n w[n][k] * dy[b][n] in fp64 (the transposed product W^T dy of the STE
+    backward, [Metal-8B]) and A[b][k] = sum_n |w[n][k] * dy[b][n]|; `cols` selects output columns.
+
+    codes: uint8 [N][stride]; scales: fp16 [N][>=K/128]; dy: fp16 [B][N].
+    """
+    t = unpack(codes, layout, k)
+    w = dequantize(t, np.asarray(scales, dtype=np.float16))
+    if cols is not None:
+        w = w[:, np.asarray(cols)]
+    dyd = np.asarray(dy, dtype=np.float16).astype(np.float64)
+    return dyd @ w, np.abs(dyd) @ np.abs(w)
 
 
 def gemm(codes, scales, X, layout: int, k: int, rows=None):

@@ -155,3 +155,28 @@ def test_hadamard_rotate_rejects_before_launch(lib):
     assert f(P(FAKE), 1, 0, P(FAKE), P(FAKE), None) == 1
     assert f(P(FAKE + 1), 1, 1024, P(FAKE), P(FAKE), None) == 3
     assert f(P(FAKE), 1, 1024, P(FAKE), P(FAKE + 1), None) == 3
+
+
+def test_pack_flips_rejects_before_launch(lib):
+    P = lambda v: ctypes.c_void_p(v)
+    f = lib.tern_pack_flips
+    ok = (1, 4, 128, P(FAKE), 128, P(FAKE + 4096), 8, P(FAKE + 8192), 32)
+    assert f(*ok, None, 32, P(FAKE + 16384), None) == 1                       # no previous codes
+    assert f(*ok, P(FAKE + 12288), 32, None, None) == 1                       # no counter
+    assert f(*ok, P(FAKE + 8192), 32, P(FAKE + 16384), None) == 1             # previous == output
+    assert f(*ok, P(FAKE + 12288), 16, P(FAKE + 16384), None) == 1            # short previous stride
+    assert f(*ok, P(FAKE + 12296), 32, P(FAKE + 16384), None) == 3            # misaligned previous codes
+    assert f(*ok, P(FAKE + 12288), 32, P(FAKE + 16388), None) == 3            # misaligned counter
+
+
+def test_gemv_t_rejects_before_launch(lib):
+    P = lambda v: ctypes.c_void_p(v)
+    m = _mat(n=4096, k=4096, code_row_stride=1024, scale_row_stride=32)
+    need = lib.tern_gemv_t_workspace_bytes(ctypes.byref(m), 1)
+    assert need > 0 and need % 4 == 0
+    assert lib.tern_gemv_t_workspace_bytes(ctypes.byref(m), 9) == 0
+    assert lib.tern_gemv_t(ctypes.byref(m), P(FAKE), 9, P(FAKE), None, 0, None) == 1
+    assert lib.tern_gemv_t(ctypes.byref(m), None, 1, P(FAKE), None, 0, None) == 1
+    assert lib.tern_gemv_t(ctypes.byref(m), P(FAKE + 1), 1, P(FAKE), None, 0, None) == 3
+    assert lib.tern_gemv_t(ctypes.byref(m), P(FAKE), 1, P(FAKE), None, 0, None) == 4
+    assert lib.tern_gemv_t(ctypes.byref(m), P(FAKE), 1, P(FAKE), P(FAKE + 8), need, None) == 3

@@ -114,3 +114,27 @@ def test_unpack_counts_invalid_codes(layout):
         inv = codes[:, kk // 5] > 242
     ref[inv] = 0
     assert np.array_equal(tt.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("layout", [T.Q2_0_G128, T.T3_5PB_G128])
+@pytest.mark.parametrize("n,k", [(257, 640), (4096, 4096)])
+def test_pack_flips_match_oracle(layout, n, k):
+    # QAT step: re-pack perturbed latents against the previous packing and count the changed codes
+    t = synth.ternary_codes(n, k, seed=n + k)
+    s = synth.group_scales(n, k // 128, seed=n + k)
+    w1 = synth.latents(t, s, seed=1)
+    w2 = (w1.astype(np.float32) + np.random.default_rng(2).standard_normal(w1.shape).astype(np.float32)
+          * 0.2 * np.repeat(s.astype(np.float32), 128, axis=1)).astype(np.float16)
+    sg = torch.from_numpy(s).cuda()
+    W1 = T.pack(torch.from_numpy(w1).cuda(), sg, layout)
+    W2, flips = T.pack_flips(torch.from_numpy(w2).cuda(), sg, W1)
+    torch.cuda.synchronize()
+    c1, c2 = W1.codes.cpu().numpy(), W2.codes.cpu().numpy()
+    assert np.array_equal(c2, O.pack(O.ternarize(w2, s), layout))  # the pack itself is unchanged
+    want = O.count_flips(c1, c2, layout, k)
+    assert int(flips.item()) == want
+    assert want == int((O.ternarize(w1, s) != O.ternarize(w2, s)).sum())
+    # the counter accumulates
+    T.pack_flips(torch.from_numpy(w2).cuda(), sg, W1, flips=flips)
+    torch.cuda.synchronize()
+    assert int(flips.item()) == 2 * want

@@ -358,3 +358,53 @@ def test_planted_mistakes_are_caught():
     assert np.allclose(O.gemv(p, sc, x, O.Q2_0_G128, k)[0], ex, rtol=1e-12, atol=0)
     assert not np.allclose(_gemv_scale_dropped(p, sc, x, O.Q2_0_G128, k), ex, rtol=1e-3)
     assert not np.allclose(_gemv_scale_wrong_group(p, sc, x, O.Q2_0_G128, k), ex, rtol=1e-3)
+
+
+@pytest.mark.parametrize("layout", [O.Q2_0_G128, O.T3_5PB_G128])
+def test_count_flips_pins(layout):
+    k = 640
+    t1 = synth.ternary_codes(40, k, seed=11)
+    p1 = O.pack(t1, layout)
+    assert O.count_flips(p1, p1, layout, k) == 0
+    # any set of changed weights: the count is the number of changed t (unpack is an independent read)
+    t2 = t1.copy()
+    rng = np.random.default_rng(12)
+    for _ in range(37):
+        r, c = rng.integers(0, 40), rng.integers(0, k)
+        t2[r, c] = (t2[r, c] + 2) % 3 - 1  # -1 -> 0 -> 1 -> -1
+    p2 = O.pack(t2, layout)
+    assert O.count_flips(p1, p2, layout, k) == int((O.unpack(p1, layout, k) != O.unpack(p2, layout, k)).sum())
+    assert O.count_flips(p1, p2, layout, k) == int((t1 != t2).sum())
+    assert O.count_flips(p1, p2, layout, k) == O.count_flips(p2, p1, layout, k)
+
+
+def test_count_flips_ignores_base3_padding():
+    k = 128  # 26 bytes of trits (128 = 25*5 + 3), byte 25 holds 2 padding trits
+    t = synth.ternary_codes(3, k, seed=13)
+    p = O.pack(t, O.T3_5PB_G128)
+    q = p.copy()
+    q[:, 25] = (q[:, 25] % 27) + 27 * 2  # change only the digits of the padding trits (k = 128, 129)
+    assert O.count_flips(p, q, O.T3_5PB_G128, k) == 0
+    q[:, 30] = 0  # a byte past the data
+    assert O.count_flips(p, q, O.T3_5PB_G128, k) == 0
+
+
+@pytest.mark.parametrize("layout", [O.Q2_0_G128, O.T3_5PB_G128])
+def test_transposed_product_is_the_adjoint(layout):
+    # <dx, x> = <dy, W x> for every x, dy: W^T is the adjoint of the forward product (checked with the
+    # forward oracle), and integer inputs give exact integers
+    n, k = 37, 640
+    t = synth.ternary_codes(n, k, seed=21)
+    codes = O.pack(t, layout)
+    s = synth.group_scales(n, k // 128, seed=21)
+    rng = np.random.default_rng(22)
+    x = rng.integers(-3, 4, size=(1, k)).astype(np.float16)
+    dy = rng.integers(-3, 4, size=(2, n)).astype(np.float16)
+    dx, _ = O.gemv_t(codes, s, dy, layout, k)
+    y, _ = O.gemv(codes, s, x, layout, k)
+    for b in range(2):
+        assert math.isclose(float(dx[b] @ x[0].astype(np.float64)), float(y[0] @ dy[b].astype(np.float64)),
+                            rel_tol=1e-12, abs_tol=1e-9)
+    ones = np.ones((n, k // 128), dtype=np.float16)
+    dxi, _ = O.gemv_t(codes, ones, dy, layout, k)
+    assert np.array_equal(dxi, dy.astype(np.int64) @ t.astype(np.int64))
