@@ -53,8 +53,8 @@ def parse():
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--no-extras", action="store_true", help="skip the per-row measurements of the other kernels")
     p.add_argument("--profile", default=None, metavar="CASE",
-                   help="run a few launches of one kernel case for ncu: gemv_{q2|t3}_NxK_bB, gemm_q2_MxNxK, "
-                        "pack_{q2|t3}_NxK")
+                   help="run a few launches of one kernel case for ncu: gemv_{q2|t3|q1}_NxK_bB, "
+                        "gemm_{q2|t3|q1}_MxNxK, pack_{q2|t3|q1}_NxK")
     return p.parse_args()
 
 
@@ -373,8 +373,8 @@ def measure_extras(torch, T, dev, peaks, stream):
         del g
         return a.elapsed_time(b) / reps
 
-    # ternarize + pack of fp16 latents, 8B shapes (both layouts)
-    for layout, name in ((T.Q2_0_G128, "q2"), (T.T3_5PB_G128, "t3")):
+    # ternarize (binarize) + pack of fp16 latents, 8B shapes (every layout)
+    for layout, name in ((T.Q2_0_G128, "q2"), (T.T3_5PB_G128, "t3"), (T.Q1_0_G128, "q1")):
         tot_b, tot_ms = 0, 0.0
         for (n, k) in LAYER_SET:
             w = torch.randn((n, k), device=dev).mul_(0.02).to(torch.float16)
@@ -390,6 +390,10 @@ def measure_extras(torch, T, dev, peaks, stream):
 
     # LM head (base-3) and 27B batched GEMVs; weights larger than L2, re-read each launch
     cases = [("lm_head_t3", T.T3_5PB_G128, 151936, 4096, b) for b in (1, 8)]
+    # the binary layout on the 8B shapes: batch 1-2 is one launch, larger batches one launch per pair
+    for (n, k) in LAYER_SET:
+        for b in (1, 2, 4, 16):
+            cases.append((f"8b_q1_{n}x{k}", T.Q1_0_G128, n, k, b))
     for layout, lname in ((T.Q2_0_G128, "q2"), (T.T3_5PB_G128, "t3")):
         for (n, k) in ((34816, 5120), (5120, 17408)):
             for b in (1, 4, 16, 64):
@@ -400,7 +404,10 @@ def measure_extras(torch, T, dev, peaks, stream):
         if key not in cache:
             cache.clear()
             torch.cuda.empty_cache()
-            cache[key] = [make_weights(torch, T, n, k, layout, 77 + c, dev) for c in range(2 if n * k > 1e8 else 6)]
+            # enough weight copies that one pass over them is over twice the 126 MB L2
+            wbytes = n * T.row_bytes(layout, k) + n * (k // GROUP) * 2
+            copies = max(2, min(64, -(-300_000_000 // wbytes)))
+            cache[key] = [make_weights(torch, T, n, k, layout, 77 + c, dev) for c in range(copies)]
         Ws = cache[key]
         x = torch.randn((b, k), device=dev).to(torch.float16)
         y = torch.empty((b, n), dtype=torch.float16, device=dev)
@@ -421,7 +428,7 @@ def measure_extras(torch, T, dev, peaks, stream):
     torch.cuda.empty_cache()
 
     # transposed product dx = W^T dy (STE backward) on the 8B shapes, batch 1
-    for layout, lname in ((T.Q2_0_G128, "q2"), (T.T3_5PB_G128, "t3")):
+    for layout, lname in ((T.Q2_0_G128, "q2"), (T.T3_5PB_G128, "t3"), (T.Q1_0_G128, "q1")):
         for (n, k) in ((24576, 4096), (4096, 12288)):
             Wt = make_weights(torch, T, n, k, layout, 6, dev)
             dy = torch.randn((1, n), device=dev).to(torch.float16)
@@ -450,7 +457,7 @@ def measure_extras(torch, T, dev, peaks, stream):
     M, N, K = 2048, 17408, 5120
     X = torch.randn((M, K), device=dev).to(torch.float16)
     Y = torch.empty((M, N), dtype=torch.float16, device=dev)
-    for layout, lname in ((T.Q2_0_G128, "q2"), (T.T3_5PB_G128, "t3")):
+    for layout, lname in ((T.Q2_0_G128, "q2"), (T.T3_5PB_G128, "t3"), (T.Q1_0_G128, "q1")):
         key = f"gemm_{lname}_2048x17408x5120"
         try:
             Wg = make_weights(torch, T, N, K, layout, 5, dev)
@@ -554,7 +561,7 @@ def run_profile_case(case: str, launches: int = 6):
     import gemm_tern_gemv_b200 as T
     dev = torch.device("cuda", 0)
     parts = case.split("_")
-    kind, layout = parts[0], (T.Q2_0_G128 if parts[1] == "q2" else T.T3_5PB_G128)
+    kind, layout = parts[0], {"q2": T.Q2_0_G128, "t3": T.T3_5PB_G128, "q1": T.Q1_0_G128}[parts[1]]
     if kind == "gemv":
         n, k = (int(v) for v in parts[2].split("x"))
         b = int(parts[3][1:])

@@ -16,6 +16,7 @@ from dataclasses import dataclass
 
 Q2_0_G128 = 1
 T3_5PB_G128 = 2
+Q1_0_G128 = 3
 GROUP = 128
 GEMV_MAX_BATCH = 64
 DEVICE_TIMEOUT = 1

@@ -14,6 +14,7 @@ int64_t row_bytes(int32_t layout, int64_t k) {
   int64_t b;
   if (layout == TERN_Q2_0_G128) b = k / 4;           // 4 two-bit codes per byte
   else if (layout == TERN_T3_5PB_G128) b = (k + 4) / 5;  // 5 trits per byte
+  else if (layout == TERN_Q1_0_G128) b = k / 8;      // 8 sign bits per byte
   else return -1;
   return (b + 15) / 16 * 16;
 }
@@ -38,11 +39,14 @@ int sm_count() {
 using namespace tern;
 
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static inline bool valid_layout(int32_t l) {
+  return l == TERN_Q2_0_G128 || l == TERN_T3_5PB_G128 || l == TERN_Q1_0_G128;
+}
 
 // Checks shared by every call that takes a packed matrix.
 static tern_status check_matrix(const tern_matrix* W) {
   if (!W) return TERN_ERR_INVALID_ARG;
-  if (W->layout != TERN_Q2_0_G128 && W->layout != TERN_T3_5PB_G128) return TERN_ERR_UNSUPPORTED;
+  if (!valid_layout(W->layout)) return TERN_ERR_UNSUPPORTED;
   if (W->n <= 0 || W->k <= 0 || W->k % kGroup) return TERN_ERR_INVALID_ARG;
   if (W->n > (int64_t)INT32_MAX || W->k > (int64_t)INT32_MAX / 2) return TERN_ERR_INVALID_ARG;
   if (!W->codes || !W->scales) return TERN_ERR_INVALID_ARG;
@@ -75,7 +79,7 @@ static tern_status pack_common(int32_t layout, int64_t n, int64_t k, const uint1
                                const uint16_t* scales, int64_t scale_row_stride, void* codes,
                                int64_t code_row_stride, const void* prev, int64_t prev_row_stride,
                                uint64_t* flips, void* stream) {
-  if (layout != TERN_Q2_0_G128 && layout != TERN_T3_5PB_G128) return TERN_ERR_UNSUPPORTED;
+  if (!valid_layout(layout)) return TERN_ERR_UNSUPPORTED;
   if (n <= 0 || k <= 0 || k % kGroup || n > (int64_t)INT32_MAX || k > (int64_t)INT32_MAX / 2)
     return TERN_ERR_INVALID_ARG;
   if (!w || !scales || !codes) return TERN_ERR_INVALID_ARG;
@@ -125,7 +129,7 @@ tern_status tern_unpack(const tern_matrix* W, uint16_t* w_out, int64_t w_row_str
 
 size_t tern_gemv_workspace_bytes(const tern_matrix* W, int64_t batch) {
   if (!W || W->n <= 0 || W->k <= 0 || W->k % kGroup) return 0;
-  if (W->layout != TERN_Q2_0_G128 && W->layout != TERN_T3_5PB_G128) return 0;
+  if (!valid_layout(W->layout)) return 0;
   if (batch < 1 || batch > TERN_GEMV_MAX_BATCH) return 0;
   return gemv_plan(W->layout, W->n, W->k, batch, sm_count()).ws_bytes;
 }
@@ -136,6 +140,7 @@ tern_status tern_gemv(const tern_matrix* W, const uint16_t* x, int64_t batch, ui
   if (s != TERN_OK) return s;
   if (batch < 1 || batch > TERN_GEMV_MAX_BATCH || !x || !y) return TERN_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y)) return TERN_ERR_ALIGNMENT;
+  if (!gemv_supported(W->layout, W->n, W->k, batch)) return TERN_ERR_UNSUPPORTED;
   GemvPlan plan = gemv_plan(W->layout, W->n, W->k, batch, sm_count());
   if (plan.ws_bytes) {
     if (!workspace || workspace_bytes < plan.ws_bytes) return TERN_ERR_WORKSPACE;
@@ -149,6 +154,7 @@ tern_status tern_gemv_noalloc(const tern_matrix* W, const uint16_t* x, int64_t b
   if (s != TERN_OK) return s;
   if (batch < 1 || batch > TERN_GEMV_MAX_BATCH || !x || !y) return TERN_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y)) return TERN_ERR_ALIGNMENT;
+  if (!gemv_supported(W->layout, W->n, W->k, batch)) return TERN_ERR_UNSUPPORTED;
   return gemv_noalloc(*W, x, (int)batch, y, static_cast<cudaStream_t>(stream));
 }
 
@@ -165,7 +171,7 @@ tern_status tern_gemm(const tern_matrix* W, const uint16_t* X, int64_t m, uint16
 
 size_t tern_gemv_t_workspace_bytes(const tern_matrix* W, int64_t batch) {
   if (!W || W->n <= 0 || W->k <= 0 || W->k % kGroup) return 0;
-  if (W->layout != TERN_Q2_0_G128 && W->layout != TERN_T3_5PB_G128) return 0;
+  if (!valid_layout(W->layout)) return 0;
   if (batch < 1 || batch > TERN_GEMV_T_MAX_BATCH) return 0;
   return gemv_t_plan(W->layout, W->n, W->k, batch, sm_count()).ws_bytes;
 }

@@ -6,7 +6,8 @@
 //
 //   * One persistent CTA per SM walks 128 (weight rows) x 256 (tokens) output tiles.
 //   * TMA streams, per 64-wide K block, the fp16 X tile (256 x 64, 128-byte swizzle) and the packed
-//     Q2_0_g128 codes of the W tile (128 rows x 16 bytes) into a 4-stage ring.
+//     codes of the W tile (128 rows x 16 bytes for Q2_0_g128 and the binary Q1_0_g128, 32 for
+//     base-3) into a 4-stage ring.
 //   * Four decoder warps expand the codes to fp16 2*s*t (exact) straight into the K-major
 //     128-byte-swizzled shared-memory layout a tcgen05 descriptor reads; a K block lies inside one
 //     128-weight group, so one scale per row and block.
@@ -41,9 +42,10 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
 constexpr int X_STAGE_BYTES = BN * BK * 2;      // 32 KB
 constexpr int A_STAGE_BYTES = BM * BK * 2;      // 16 KB
 // Packed codes of a K block, per row: Q2_0_g128 16 bytes; base-3 a 32-byte box at the 16-byte
-// boundary below the block's first byte (the block's 64 trits span at most 14 bytes).
-template <int LAYOUT> constexpr int p_row_bytes() { return LAYOUT == TERN_Q2_0_G128 ? BK / 4 : 32; }
-constexpr int P_STAGE_BYTES = BM * 32;          // room for either layout
+// boundary below the block's first byte (the block's 64 trits span at most 14 bytes); binary the
+// 16-byte box holding the block's 8 bytes (TMA boxes start on 16-byte boundaries).
+template <int LAYOUT> constexpr int p_row_bytes() { return LAYOUT == TERN_T3_5PB_G128 ? 32 : 16; }
+constexpr int P_STAGE_BYTES = BM * 32;          // room for any layout
 constexpr int OFF_X = 0;
 constexpr int OFF_A = OFF_X + STAGES * X_STAGE_BYTES;
 constexpr int OFF_P = OFF_A + DSTAGES * A_STAGE_BYTES;
@@ -71,6 +73,14 @@ __device__ __forceinline__ uint32_t pair_2t(uint32_t w, int j) {
   const uint32_t x = lo & (0xFu << (4 * jj));
   const uint32_t a = 14 - 4 * jj;  // field 2j (bits 4jj..) -> bit 14; field 2j+1 -> bit 30
   return (x * ((1u << a) + (1u << (a + 14)))) & 0xC000C000u;
+}
+
+// Binary sign bits (bit i of w = weight i, 1 = +1) -> fp16 pair (2 t_p, 2 t_{p+1}) for an even
+// p <= 14: one multiply moves bit p to bit 15 and bit p + 1 to bit 31, and flipping the sign and the
+// exponent MSB turns a set sign bit into +2.0 (0x4000) and a clear one into -2.0 (0xC000).
+__device__ __forceinline__ uint32_t pair_2t_bin(uint32_t w, int p) {
+  const uint32_t x = w & (3u << p);
+  return ((x * ((1u << (15 - p)) + (1u << (30 - p)))) & 0x80008000u) ^ 0xC000C000u;
 }
 
 // Base-3 K block whose first trit is digit R0 of its first byte: the 64 weights -> fp16 2 s t in the
@@ -172,7 +182,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
           }
           mbar_arrive_expect_tx(full + s, X_STAGE_BYTES + BM * p_row_bytes<LAYOUT>());
           tma_load_2d(smem + OFF_X + s * X_STAGE_BYTES, &tmap_x, full + s, kb * BK, m0);
-          const int px = LAYOUT == TERN_Q2_0_G128 ? kb * (BK / 4) : ((kb * BK) / 5) & ~15;
+          const int px = LAYOUT == TERN_Q2_0_G128 ? kb * (BK / 4)
+                         : LAYOUT == TERN_Q1_0_G128 ? (kb * (BK / 8)) & ~15
+                                                    : ((kb * BK) / 5) & ~15;
           tma_load_2d(smem + OFF_P + s * P_STAGE_BYTES, &tmap_w, full + s, px, n0);
           pending[s] = true;
           pend_par[s] = ph;
@@ -289,6 +301,21 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             }
             *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
           }
+        } else if (LAYOUT == TERN_Q1_0_G128) {
+          // the block's 8 bytes are the low or high half of the 16-byte box
+          const uint2 pk = *reinterpret_cast<const uint2*>(smem + OFF_P + s * P_STAGE_BYTES + r * 16 + 8 * (kb & 1));
+#pragma unroll
+          for (int c = 0; c < 8; c++) {  // byte c holds k = 8c .. 8c + 7
+            const uint32_t w = (c < 4 ? pk.x : pk.y) >> (c & 2 ? 16 : 0);
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+              const uint32_t two_t = pair_2t_bin(w, 8 * (c & 1) + 2 * e);
+              const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&two_t), s2);  // 2 s t, exact
+              o[e] = *reinterpret_cast<const uint32_t*>(&v);
+            }
+            *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          }
         } else {
           // the block's trits start at digit r0 of byte b0; the box starts at the 16-byte boundary below b0
           const int b0 = (kb * BK) / 5, r0 = (kb * BK) % 5;
@@ -323,12 +350,14 @@ cudaError_t launch_gemm(const tern_matrix& W, const uint16_t* X, int64_t m, uint
                         cudaStream_t st) {
   CUtensorMap mx, mw;
   const uint64_t k = (uint64_t)W.k, n = (uint64_t)W.n;
-  const bool q2 = W.layout == TERN_Q2_0_G128;
+  const bool t3 = W.layout == TERN_T3_5PB_G128;
   if (!tmap_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, X, k, (uint64_t)m, k * 2, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  // codes [n][row data bytes]: Q2 boxes of 16 bytes, base-3 boxes of 32 bytes (zero-filled past the data)
-  if (!tmap_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.codes, q2 ? k / 4 : (k + 4) / 5, n, (uint64_t)W.code_row_stride,
-               q2 ? BK / 4 : 32, BM, CU_TENSOR_MAP_SWIZZLE_NONE))
+  // codes [n][row data bytes]: Q2 and binary boxes of 16 bytes, base-3 boxes of 32 bytes (zero-filled
+  // past the data)
+  const uint64_t data_bytes = W.layout == TERN_Q2_0_G128 ? k / 4 : W.layout == TERN_Q1_0_G128 ? k / 8 : (k + 4) / 5;
+  if (!tmap_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.codes, data_bytes, n, (uint64_t)W.code_row_stride,
+               t3 ? 32 : 16, BM, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   Params p;
   p.m = (int)m;
@@ -340,7 +369,9 @@ cudaError_t launch_gemm(const tern_matrix& W, const uint16_t* X, int64_t m, uint
   p.sstride = W.scale_row_stride;
   p.y = Y;
   p.status = device_status;
-  auto kern = q2 ? gemm_kernel<TERN_Q2_0_G128> : gemm_kernel<TERN_T3_5PB_G128>;
+  auto kern = W.layout == TERN_Q2_0_G128   ? gemm_kernel<TERN_Q2_0_G128>
+              : W.layout == TERN_Q1_0_G128 ? gemm_kernel<TERN_Q1_0_G128>
+                                           : gemm_kernel<TERN_T3_5PB_G128>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int tiles = p.n_tiles * p.m_tiles;

@@ -119,6 +119,13 @@ __device__ __forceinline__ void mma_f16_first(float* d, uint32_t a0, uint32_t a1
 // `mul` is 2^(14 - 2S) held in a register, so the shift issues as an IMAD on the FMA pipe.
 __device__ __forceinline__ uint32_t slot(uint32_t w, uint32_t mul) { return (w * mul) & 0xC000C000u; }
 
+// Binary A fragment of slot S (0..15) of a 32-bit word of sign bits: bits (S, S+16) as the fp16 pair
+// (2 t_S, 2 t_S+16). `mul` = 2^(15 - S) moves the bits to the two sign positions; flipping sign and
+// exponent MSB then gives +2.0 (0x4000) for a set bit and -2.0 (0xC000) for a clear one.
+__device__ __forceinline__ uint32_t slot_bin(uint32_t w, uint32_t mul) {
+  return ((w * mul) & 0x80008000u) ^ 0xC000C000u;
+}
+
 // ---- shared-memory plan (host and device agree on it) -------------------------------------------
 __host__ __device__ inline int pair_windows(int layout, int gps) {
   return layout == TERN_T3_5PB_G128 ? 3 * ((gps + kT3Window - 1) / kT3Window) : (gps + 1) / 2;
@@ -570,12 +577,14 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(Args a) {
   cp_async_wait<0>();
 }
 
-// ---- small batches: both layouts decoded in registers ----------------------------------------------
-// One window = 64 code bytes of every row of a warp tile: 256 weights (two groups) of Q2_0_g128 or
-// 320 weights of the base-3 layout. Lane (g, q) owns bytes [16q, 16q + 16) of rows g and g + 8 of
+// ---- small batches: every layout decoded in registers -----------------------------------------------
+// One window = 64 code bytes of every row of a warp tile: 256 weights (two groups) of Q2_0_g128,
+// 320 weights of the base-3 layout or 512 weights (four groups) of the binary Q1_0_g128. Lane (g, q) owns bytes [16q, 16q + 16) of rows g and g + 8 of
 // each 16-row tile, decodes them straight into mma.sync A fragments and never writes codes back to
 // shared memory:
 //   * Q2_0_g128: slot S of a 16-code word is (word * 2^(14 - 2S)) & 0xC000C000 (see slot()).
+//   * Q1_0_g128: slot S of a 32-bit word is bits (S, S + 16) placed as two signs (see slot_bin());
+//     a lane's 16 bytes are exactly one group.
 //   * base-3: bytes (0, 2) and (1, 3) of a word sit in 16-bit lanes V; with c = t + 1 the five digits
 //     come out most significant first from one multiply-add and a chain of "times three" steps:
 //     R = V * 202 + 130 maps each byte v to r = floor(R / 64) in [256 v / 81, 256 (v + 1) / 81), so
@@ -586,6 +595,7 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(Args a) {
 //     masked or already garbage); an invalid byte (> 242) gives unspecified trits.
 // The MMA columns are (batch, group-within-window) pairs: a base-3 window touches three groups, so a
 // lane's four k-slots may belong to two groups and the activation fragments are stored per column.
+// A binary window holds four groups, so its eight columns carry two batch rows.
 #ifndef TERN_REG_WARPS
 #define TERN_REG_WARPS 16
 #endif
@@ -610,15 +620,25 @@ template <> struct Lay<TERN_T3_5PB_G128> {
   static constexpr int SC = 2;
   static constexpr int W = 320;
 };
+template <> struct Lay<TERN_Q1_0_G128> {
+  static constexpr int J = 32;
+  static constexpr int C = 1;    // the lane's group is q
+  static constexpr int SC = 1;
+  static constexpr int W = 512;
+};
 
 __host__ __device__ inline int s_windows(int layout, int ngroups) {
-  return layout == TERN_Q2_0_G128 ? (ngroups + 1) / 2 : (ngroups * kGroup + 319) / 320;
+  return layout == TERN_Q2_0_G128   ? (ngroups + 1) / 2
+         : layout == TERN_Q1_0_G128 ? (ngroups + 3) / 4
+                                    : (ngroups * kGroup + 319) / 320;
 }
 __host__ __device__ constexpr uint32_t s_frag_window_bytes(int layout, int bs) {
-  return layout == TERN_Q2_0_G128 ? 8u * bs * 1 * 4 * 16 : 10u * bs * 3 * 4 * 16;
+  return layout == TERN_Q2_0_G128   ? 8u * bs * 1 * 4 * 16
+         : layout == TERN_Q1_0_G128 ? 16u * bs * 1 * 4 * 16
+                                    : 10u * bs * 3 * 4 * 16;
 }
 __host__ __device__ constexpr uint32_t s_stage_bytes(int layout, int rt) {
-  return (uint32_t)rt * 16 * (kWinBytes + 16 * (layout == TERN_Q2_0_G128 ? 1 : 2));
+  return (uint32_t)rt * 16 * (kWinBytes + 16 * (layout == TERN_T3_5PB_G128 ? 2 : 1));
 }
 __host__ __device__ inline size_t s_smem_bytes(int layout, int rt, int stages, int gps, int bs) {
   return (size_t)s_frag_window_bytes(layout, bs) * (s_windows(layout, gps) + 1) +
@@ -663,7 +683,7 @@ __device__ __forceinline__ void dec_t3_word(uint32_t w, uint32_t k0, uint32_t (&
 template <int LAYOUT, int BS, int HF>
 __device__ __forceinline__ void s_frag_half(const Args& a, int g0, int kslice, int w, int q, int b, uint16_t* fh) {
   using L = Lay<LAYOUT>;
-  constexpr int HW = L::W / 8;  // weights of a lane chunk half: 32 (Q2) or 40 (base-3)
+  constexpr int HW = L::W / 8;  // weights of a lane chunk half: 32 (Q2), 40 (base-3) or 64 (binary)
   const int k0 = w * L::W + (L::W / 4) * q + HF * HW;  // first weight within the slice
   const uint16_t* xs = a.x + (int64_t)b * a.k + (int64_t)g0 * kGroup + k0;
   uint32_t xw[HW / 2];
@@ -682,6 +702,10 @@ __device__ __forceinline__ void s_frag_half(const Args& a, int g0, int kslice, i
       const int word = c >> 4, i = c & 15, S = i & 7;
       j = 4 * word + (S >> 1);
       e4 = 2 * (S & 1) + (i >> 3);
+    } else if (LAYOUT == TERN_Q1_0_G128) {
+      const int word = c >> 5, i = c & 31, S = i & 15;
+      j = 8 * word + (S >> 1);
+      e4 = 2 * (S & 1) + (i >> 4);
     } else {
       const int bl = c / 5, d = c - 5 * bl, word = bl >> 2, bb = bl & 3;
       const int r = 5 * (bb & 1) + (4 - d);
@@ -698,7 +722,7 @@ template <int LAYOUT, int BS>
 __device__ void s_build_frag(const Args& a, int g0, int ngroups, int nwin_alloc, uint8_t* frag) {
   constexpr uint32_t FW = s_frag_window_bytes(LAYOUT, BS);
   uint4* f4 = reinterpret_cast<uint4*>(frag);
-  if (LAYOUT == TERN_Q2_0_G128) {
+  if (LAYOUT != TERN_T3_5PB_G128) {
     // every entry a data lane reads is written below (zero past the slice); only the zero block
     for (int i = threadIdx.x; i < (int)(FW / 16); i += kSThreads)
       f4[(size_t)nwin_alloc * FW / 16 + i] = make_uint4(0u, 0u, 0u, 0u);
@@ -738,14 +762,14 @@ __device__ __forceinline__ int s_contributors(const Args& a, int tile) {  // run
   return c;
 }
 
-// Lane (g, q) accumulates rows g, g + 8 of each 16-row tile. Q2: lane q holds batch q. Base-3: lanes
-// q and q ^ 1 hold batch q / 2 (groups 0-1 and 2 of each window) and are summed here; the even lane
-// of the pair stores.
+// Lane (g, q) accumulates rows g, g + 8 of each 16-row tile. Q2: lane q holds batch q. Base-3 and
+// binary: lanes q and q ^ 1 hold batch q / 2 (base-3: groups 0-1 and 2 of each window; binary: groups
+// 0-1 and 2-3) and are summed here; the even lane of the pair stores.
 template <int LAYOUT, int RT>
 __device__ __forceinline__ void s_combine(float (&acc)[RT][2], int& b, bool& owner, int q) {
   b = q;
   owner = true;
-  if (LAYOUT == TERN_T3_5PB_G128) {
+  if (LAYOUT != TERN_Q2_0_G128) {
 #pragma unroll
     for (int rt = 0; rt < RT; rt++)
 #pragma unroll
@@ -876,12 +900,16 @@ __global__ void __launch_bounds__(kSThreads, kRegCtasPerSm)
 
   // ---- issue side (lane 0): one TMA box of codes [ROWS][64 B] and one of scales per window; reads
   // past the row data, the scale columns or the last row are zero-filled by the tensor maps
-  const int slice_x0 = LAYOUT == TERN_Q2_0_G128 ? g0 * (kGroup / 4) : (g0 / 5) * 128;
+  const int slice_x0 = LAYOUT == TERN_Q2_0_G128   ? g0 * (kGroup / 4)
+                       : LAYOUT == TERN_Q1_0_G128 ? g0 * (kGroup / 8)
+                                                  : (g0 / 5) * 128;
   int is_tile = tile0, is_w = w0, is_slot = 0;
   auto issue_next = [&]() {
     uint64_t* bar = full + is_slot;
     uint8_t* dst = ring + is_slot * STAGE;
-    const int gfirst = LAYOUT == TERN_Q2_0_G128 ? g0 + 2 * is_w : g0 + (5 * is_w) / 2;
+    const int gfirst = LAYOUT == TERN_Q2_0_G128   ? g0 + 2 * is_w
+                       : LAYOUT == TERN_Q1_0_G128 ? g0 + 4 * is_w
+                                                  : g0 + (5 * is_w) / 2;
     sm100::mbar_arrive_expect_tx(bar, STAGE);
     sm100::tma_load_2d(dst, &tm_codes, bar, slice_x0 + kWinBytes * is_w, is_tile * ROWS);
     sm100::tma_load_2d(dst + kCodeBytes, &tm_scales, bar, 8 * (gfirst >> 3), is_tile * ROWS);
@@ -901,6 +929,8 @@ __global__ void __launch_bounds__(kSThreads, kRegCtasPerSm)
   bool fdata;
   if (LAYOUT == TERN_Q2_0_G128) {
     fb = g >> 1; fcol = 0; fdata = ((g & 1) == (q >> 1)) && fb < a.batch;
+  } else if (LAYOUT == TERN_Q1_0_G128) {
+    fb = g >> 2; fcol = 0; fdata = ((g & 3) == q) && fb < a.batch;
   } else {
     fb = g >> 2; fcol = g & 3; fdata = fcol < 3 && fb < a.batch;
   }
@@ -908,9 +938,11 @@ __global__ void __launch_bounds__(kSThreads, kRegCtasPerSm)
                                : smem_u32(frag) + (uint32_t)nwin_alloc * FW;
   const uint32_t fstep = fdata ? FW : 0u;
 
-  uint32_t mul[8];
+  uint32_t mul[8], mulb[16];
 #pragma unroll
   for (int S = 0; S < 8; S++) mul[S] = a.unit << (14 - 2 * S);
+#pragma unroll
+  for (int S = 0; S < 16; S++) mulb[S] = a.unit << (15 - S);
   const uint32_t k0 = a.unit * (130u | (130u << 16)) + 0xC000C000u;
 
   float acc[RT][2];
@@ -935,10 +967,12 @@ __global__ void __launch_bounds__(kSThreads, kRegCtasPerSm)
     for (int rt = 0; rt < RT; rt++)
 #pragma unroll
       for (int hr = 0; hr < 2; hr++) cw[rt][hr] = lds128(stage_u + lane_code + (rt * 16 + 8 * hr) * kWinBytes);
-    // fragment pairs a word needs: Q2 word w uses pairs 2w, 2w + 1; base-3 word w uses pairs
-    // floor(5w / 2) .. floor((5w + 4) / 2)
-    constexpr int NB = LAYOUT == TERN_Q2_0_G128 ? 2 : 3;
-    auto pair0 = [](int word) { return LAYOUT == TERN_Q2_0_G128 ? 2 * word : (5 * word) >> 1; };
+    // fragment pairs a word needs: Q2 word w uses pairs 2w, 2w + 1; binary word w pairs 4w .. 4w + 3;
+    // base-3 word w pairs floor(5w / 2) .. floor((5w + 4) / 2)
+    constexpr int NB = LAYOUT == TERN_Q2_0_G128 ? 2 : LAYOUT == TERN_Q1_0_G128 ? 4 : 3;
+    auto pair0 = [](int word) {
+      return LAYOUT == TERN_Q2_0_G128 ? 2 * word : LAYOUT == TERN_Q1_0_G128 ? 4 * word : (5 * word) >> 1;
+    };
     uint4 bcur[NB], bnext[NB];
 #pragma unroll
     for (int i = 0; i < NB; i++) bcur[i] = lds128(fa + (pair0(0) + i) * kJP);
@@ -949,7 +983,27 @@ __global__ void __launch_bounds__(kSThreads, kRegCtasPerSm)
 #pragma unroll
         for (int i = 0; i < NB; i++) bnext[i] = lds128(fa + (pair0(word + 1) + i) * kJP);
       }
-      if (LAYOUT == TERN_Q2_0_G128) {
+      if (LAYOUT == TERN_Q1_0_G128) {
+        uint32_t wl[RT], wh[RT];
+#pragma unroll
+        for (int rt = 0; rt < RT; rt++) {
+          wl[rt] = word == 0 ? cw[rt][0].x : word == 1 ? cw[rt][0].y : word == 2 ? cw[rt][0].z : cw[rt][0].w;
+          wh[rt] = word == 0 ? cw[rt][1].x : word == 1 ? cw[rt][1].y : word == 2 ? cw[rt][1].z : cw[rt][1].w;
+        }
+#pragma unroll
+        for (int sp = 0; sp < 8; sp++) {
+          const int j = 8 * word + sp;
+          const uint4 bq = bcur[(j >> 1) - pair0(word)];
+          const uint32_t b0 = (j & 1) ? bq.z : bq.x, b1 = (j & 1) ? bq.w : bq.y;
+#pragma unroll
+          for (int rt = 0; rt < RT; rt++) {
+            const uint32_t a0 = slot_bin(wl[rt], mulb[2 * sp]), a2 = slot_bin(wl[rt], mulb[2 * sp + 1]);
+            const uint32_t a1 = slot_bin(wh[rt], mulb[2 * sp]), a3 = slot_bin(wh[rt], mulb[2 * sp + 1]);
+            if (j == 0) mma_f16_first(d[rt], a0, a1, a2, a3, b0, b1);
+            else mma_f16(d[rt], a0, a1, a2, a3, b0, b1);
+          }
+        }
+      } else if (LAYOUT == TERN_Q2_0_G128) {
         uint32_t wl[RT], wh[RT];
 #pragma unroll
         for (int rt = 0; rt < RT; rt++) {
@@ -998,7 +1052,9 @@ __global__ void __launch_bounds__(kSThreads, kRegCtasPerSm)
     // the two scales this lane's columns use, per row (columns without data have D = 0)
     float sa[RT][2], sb[RT][2];
     {
-      const int gfirst = LAYOUT == TERN_Q2_0_G128 ? g0 + 2 * c_w : g0 + (5 * c_w) / 2;
+      const int gfirst = LAYOUT == TERN_Q2_0_G128   ? g0 + 2 * c_w
+                         : LAYOUT == TERN_Q1_0_G128 ? g0 + 4 * c_w
+                                                    : g0 + (5 * c_w) / 2;
       const int ja = LAYOUT == TERN_Q2_0_G128 ? 0 : 2 * (q & 1);
       const uint32_t so = stage_u + lane_scale + 2 * ((gfirst & 7) + ja);
 #pragma unroll
@@ -1006,8 +1062,8 @@ __global__ void __launch_bounds__(kSThreads, kRegCtasPerSm)
 #pragma unroll
         for (int hr = 0; hr < 2; hr++) {
           const uint32_t ra = so + (rt * 16 + 8 * hr) * (16 * L::SC);
-          if (LAYOUT == TERN_Q2_0_G128) {
-            const uint32_t pr = lds32(ra);  // groups gfirst, gfirst + 1 (gfirst is even)
+          if (LAYOUT != TERN_T3_5PB_G128) {
+            const uint32_t pr = lds32(ra);  // groups gfirst + ja, gfirst + ja + 1 (an even first group)
             const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&pr));
             sa[rt][hr] = sf.x;
             sb[rt][hr] = sf.y;
@@ -1129,6 +1185,7 @@ cudaError_t launch_reg(const CUtensorMap& tc, const CUtensorMap& ts, const Args&
 #define TERN_REG_STAGES_T3 3
 #endif
 constexpr int kRegRT = TERN_REG_RT;
+constexpr int kBinChunk = 2;  // batch rows per launch of the binary register kernel
 constexpr int kRegStagesQ2 = TERN_REG_STAGES_Q2;
 constexpr int kRegStagesT3 = TERN_REG_STAGES_T3;
 
@@ -1136,21 +1193,26 @@ bool use_reg_kernel(int32_t layout, int64_t n, int64_t k, int64_t batch) {
   // (tile, window) unit indices are 32-bit
   const int64_t units = (n + 16 * kRegRT - 1) / (16 * kRegRT) * s_windows(layout, (int)(k / kGroup));
   if (units >= ((int64_t)1 << 30)) return false;
-  return layout == TERN_Q2_0_G128 ? batch <= 4 : batch <= 2;
+  // the binary layout has no other small-batch kernel: larger batches run in pairs of rows
+  return layout == TERN_Q2_0_G128 ? batch <= 4 : layout == TERN_Q1_0_G128 ? true : batch <= 2;
 }
 
 cudaError_t dispatch_reg(const tern_matrix& W, const Args& a, int grid_x, cudaStream_t st) {
   // tensor maps: codes [n][row data bytes] in boxes of 64 B x tile rows; scales [n][groups] in boxes
-  // of 8 (Q2) or 16 (base-3) groups x tile rows
-  const bool q2 = W.layout == TERN_Q2_0_G128;
-  const uint64_t data_bytes = q2 ? (uint64_t)W.k / 4 : (uint64_t)(W.k + 4) / 5;
+  // of 8 (Q2, binary) or 16 (base-3) groups x tile rows
+  const bool q2 = W.layout == TERN_Q2_0_G128, q1 = W.layout == TERN_Q1_0_G128;
+  const uint64_t data_bytes = q2 ? (uint64_t)W.k / 4 : q1 ? (uint64_t)W.k / 8 : (uint64_t)(W.k + 4) / 5;
   CUtensorMap tc, ts;
   if (!tmap_2d(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.codes, data_bytes, (uint64_t)W.n, (uint64_t)W.code_row_stride,
                kWinBytes, 16 * kRegRT, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   if (!tmap_2d(&ts, CU_TENSOR_MAP_DATA_TYPE_UINT16, W.scales, (uint64_t)(W.k / kGroup), (uint64_t)W.n,
-               (uint64_t)W.scale_row_stride * 2, q2 ? 8 : 16, 16 * kRegRT, CU_TENSOR_MAP_SWIZZLE_NONE))
+               (uint64_t)W.scale_row_stride * 2, q2 || q1 ? 8 : 16, 16 * kRegRT, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
+  if (q1) {
+    if (a.batch == 1) return launch_reg<TERN_Q1_0_G128, kRegRT, 1, kRegStagesQ2>(tc, ts, a, grid_x, st);
+    return launch_reg<TERN_Q1_0_G128, kRegRT, 2, kRegStagesQ2>(tc, ts, a, grid_x, st);
+  }
   if (q2) {
     switch (bs_for(a.batch)) {
       case 1: return launch_reg<TERN_Q2_0_G128, kRegRT, 1, kRegStagesQ2>(tc, ts, a, grid_x, st);
@@ -1170,10 +1232,12 @@ cudaError_t dispatch_reg(const tern_matrix& W, const Args& a, int grid_x, cudaSt
 static GemvPlan reg_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
   GemvPlan p{};
   p.reg = true;
+  if (layout == TERN_Q1_0_G128) batch = std::min<int64_t>(batch, kBinChunk);  // one launch per pair of rows
   const int groups = (int)(k / kGroup);
-  const int unit = (layout == TERN_T3_5PB_G128) ? kT3Window : 2;  // K-slice granularity in groups
+  // K-slice granularity in groups: one window
+  const int unit = layout == TERN_T3_5PB_G128 ? kT3Window : layout == TERN_Q1_0_G128 ? 4 : 2;
   const int units = (groups + unit - 1) / unit;
-  const int stages = layout == TERN_Q2_0_G128 ? kRegStagesQ2 : kRegStagesT3;
+  const int stages = layout == TERN_T3_5PB_G128 ? kRegStagesT3 : kRegStagesQ2;
   const int bs = bs_for(batch);
   // shared memory of one CTA when kRegCtasPerSm of them share an SM (228 KB, 1 KB reserved each)
   const size_t cap = (size_t)(228 / kRegCtasPerSm - 1) * 1024;
@@ -1208,6 +1272,11 @@ static GemvPlan reg_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, in
 // weights at a fixed rate whatever the number of tokens sharing them, which beats the mma.sync
 // kernels once a weight serves this many rows of x.
 constexpr int kGemmMinBatch = 17;
+
+bool gemv_supported(int32_t layout, int64_t n, int64_t k, int64_t batch) {
+  if (layout != TERN_Q1_0_G128) return true;
+  return (batch >= kGemmMinBatch && n % 8 == 0) || use_reg_kernel(layout, n, k, batch);
+}
 
 GemvPlan gemv_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
   if (batch >= kGemmMinBatch && n % 8 == 0) {
@@ -1264,6 +1333,18 @@ cudaError_t launch_gemv(const tern_matrix& W, const uint16_t* x, int batch, uint
   a.kmax = plan.kmax;
   a.ws = plan.ws_bytes ? static_cast<float*>(workspace) : nullptr;
   a.counters = plan.ws_bytes ? reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + plan.ws_partial_bytes) : nullptr;
+  if (plan.reg && W.layout == TERN_Q1_0_G128) {
+    // the binary kernel's MMA columns hold two batch rows: one launch per pair, in order on the stream
+    // (the split-K partials and counters of one launch are consumed before the next starts)
+    for (int b0 = 0; b0 < batch; b0 += kBinChunk) {
+      a.batch = std::min(kBinChunk, batch - b0);
+      a.x = x + (int64_t)b0 * W.k;
+      a.y = y + (int64_t)b0 * W.n;
+      const cudaError_t e = dispatch_reg(W, a, plan.grid_x, st);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
   if (plan.reg) return dispatch_reg(W, a, plan.grid_x, st);
   const int gx_hint = (plan.row_blocks + kWarps - 1) / kWarps;
   if (W.layout == TERN_Q2_0_G128) return dispatch<TERN_Q2_0_G128>(a, gx_hint, st);

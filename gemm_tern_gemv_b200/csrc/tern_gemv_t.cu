@@ -4,10 +4,10 @@
 // ternarized forward to the latent weights and the layer input).
 //
 // The contraction runs over the rows of W, so a warp reads whole rows: CTA (column block, row slice)
-// covers 64 code bytes of every row of its slice (256 columns of Q2_0_g128, 320 of base-3); thread t
-// owns byte t % 64 of rows t / 64, t / 64 + 4, ... and accumulates its 4 (or 5) columns for every
-// batch row in fp32 with s * dy formed once per row. The four row phases of a CTA are summed through
-// shared memory; row slices write fp32 partials that a second kernel sums in slice order
+// covers 64 code bytes of every row of its slice (256 columns of Q2_0_g128, 320 of base-3, 512 of
+// the binary Q1_0_g128); thread t owns byte t % 64 of rows t / 64, t / 64 + 4, ... and accumulates its
+// 4, 5 or 8 columns for every batch row in fp32 with s * dy formed once per row. The four row phases
+// of a CTA are summed through shared memory in two halving steps; row slices write fp32 partials that a second kernel sums in slice order
 // (deterministic), or the single slice stores dx directly.
 #include <cuda_fp16.h>
 
@@ -19,7 +19,10 @@ namespace {
 constexpr int kTThreads = 256;
 constexpr int kTBytes = 64;  // code bytes of a row per column block
 
-template <int LAYOUT> constexpr int cols_per_byte() { return LAYOUT == TERN_Q2_0_G128 ? 4 : 5; }
+template <int LAYOUT> constexpr int cols_per_byte() {
+  return LAYOUT == TERN_Q2_0_G128 ? 4 : LAYOUT == TERN_Q1_0_G128 ? 8 : 5;
+}
+constexpr int kPhases = kTThreads / kTBytes;
 
 template <int LAYOUT, int BATCH>
 __global__ void __launch_bounds__(kTThreads) gemv_t_kernel(const uint8_t* __restrict__ codes, int64_t cstride,
@@ -28,13 +31,13 @@ __global__ void __launch_bounds__(kTThreads) gemv_t_kernel(const uint8_t* __rest
                                                            int64_t k, int64_t rows_per_slice, float* part,
                                                            uint16_t* dx) {
   constexpr int C = cols_per_byte<LAYOUT>();
-  __shared__ float red[kTThreads / kTBytes][kTBytes * C][BATCH];
+  __shared__ float red[kPhases / 2][kTBytes * C][BATCH];
   const int t = threadIdx.x, phase = t / kTBytes, byte = t % kTBytes;
   const int64_t col0 = (int64_t)blockIdx.x * kTBytes * C + (int64_t)byte * C;  // first column of this byte
   const int64_t n0 = (int64_t)blockIdx.y * rows_per_slice;
   const int64_t n1 = n0 + rows_per_slice < n ? n0 + rows_per_slice : n;
   const int64_t byte_off = (int64_t)blockIdx.x * kTBytes + byte;
-  const int64_t data_bytes = LAYOUT == TERN_Q2_0_G128 ? k / 4 : (k + 4) / 5;
+  const int64_t data_bytes = LAYOUT == TERN_Q2_0_G128 ? k / 4 : LAYOUT == TERN_Q1_0_G128 ? k / 8 : (k + 4) / 5;
   // groups of this byte's columns (a base-3 byte can straddle two 128-column groups)
   const int64_t g_first = col0 / kGroup, g_last = (col0 + C - 1) / kGroup;
   float acc[C][BATCH];
@@ -57,6 +60,8 @@ __global__ void __launch_bounds__(kTThreads) gemv_t_kernel(const uint8_t* __rest
         if (LAYOUT == TERN_Q2_0_G128) {
           const uint32_t f = (v >> (2 * i)) & 3u;  // two's complement field; 0b10 (invalid) reads as 0
           tv = f == 1u ? 1.f : (f == 3u ? -1.f : 0.f);
+        } else if (LAYOUT == TERN_Q1_0_G128) {
+          tv = (v >> i) & 1u ? 1.f : -1.f;  // sign bit, 1 = +1
         } else {
           const uint32_t c = v % 3u;  // digit i, c = t + 1 (an invalid byte gives unspecified t)
           v /= 3u;
@@ -68,11 +73,20 @@ __global__ void __launch_bounds__(kTThreads) gemv_t_kernel(const uint8_t* __rest
       }
     }
   }
-  // sum the four row phases
+  // sum the four row phases: phases 2, 3 hand their sums to phases 0, 1, which store theirs added
+  if (phase >= kPhases / 2) {
 #pragma unroll
-  for (int i = 0; i < C; i++)
+    for (int i = 0; i < C; i++)
 #pragma unroll
-    for (int b = 0; b < BATCH; b++) red[phase][byte * C + i][b] = acc[i][b];
+      for (int b = 0; b < BATCH; b++) red[phase - kPhases / 2][byte * C + i][b] = acc[i][b];
+  }
+  __syncthreads();
+  if (phase < kPhases / 2) {
+#pragma unroll
+    for (int i = 0; i < C; i++)
+#pragma unroll
+      for (int b = 0; b < BATCH; b++) red[phase][byte * C + i][b] += acc[i][b];
+  }
   __syncthreads();
   for (int e = t; e < kTBytes * C * BATCH; e += kTThreads) {
     const int c = e / BATCH, b = e % BATCH;
@@ -80,7 +94,7 @@ __global__ void __launch_bounds__(kTThreads) gemv_t_kernel(const uint8_t* __rest
     if (b >= batch || col >= k) continue;
     float v = 0.f;
 #pragma unroll
-    for (int p = 0; p < kTThreads / kTBytes; p++) v += red[p][c][b];
+    for (int p = 0; p < kPhases / 2; p++) v += red[p][c][b];
     if (part) part[((int64_t)blockIdx.y * batch + b) * k + col] = v;
     else dx[(int64_t)b * k + col] = __half_as_ushort(__float2half_rn(v));
   }
@@ -124,7 +138,7 @@ cudaError_t dispatch_t(const tern_matrix& W, const uint16_t* dy, int batch, uint
 
 GemvTPlan gemv_t_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
   GemvTPlan p{};
-  const int64_t cols = (int64_t)kTBytes * (layout == TERN_Q2_0_G128 ? 4 : 5);
+  const int64_t cols = (int64_t)kTBytes * (layout == TERN_Q2_0_G128 ? 4 : layout == TERN_Q1_0_G128 ? 8 : 5);
   p.col_blocks = (int)((k + cols - 1) / cols);
   // about two CTAs per SM; every slice keeps at least 64 rows
   int64_t slices = (2 * (int64_t)sms + p.col_blocks - 1) / p.col_blocks;
@@ -139,6 +153,7 @@ cudaError_t launch_gemv_t(const tern_matrix& W, const uint16_t* dy, int batch, u
                           const GemvTPlan& plan, cudaStream_t st) {
   float* part = static_cast<float*>(workspace);
   if (W.layout == TERN_Q2_0_G128) return dispatch_t<TERN_Q2_0_G128>(W, dy, batch, dx, part, plan, st);
+  if (W.layout == TERN_Q1_0_G128) return dispatch_t<TERN_Q1_0_G128>(W, dy, batch, dx, part, plan, st);
   return dispatch_t<TERN_T3_5PB_G128>(W, dy, batch, dx, part, plan, st);
 }
 

@@ -49,6 +49,9 @@ struct GemvPlan {
   size_t ws_bytes;          // partials + one int32 counter per row block, rounded to 16
 };
 GemvPlan gemv_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms);
+// False only for a binary matrix too large for the register kernel's 32-bit unit indices at a batch
+// the GEMM kernel does not take.
+bool gemv_supported(int32_t layout, int64_t n, int64_t k, int64_t batch);
 
 cudaError_t launch_gemv(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y,
                         void* workspace, const GemvPlan& plan, cudaStream_t st);

@@ -1,7 +1,7 @@
-// Ternarize-and-pack and unpack kernels for both packed layouts.
+// Ternarize-and-pack and unpack kernels for the packed layouts.
 //
-// Both are HBM-streaming kernels: one thread owns one 16-byte chunk of a packed row (64 weights
-// for Q2_0_g128, 80 for base-3), reads or writes the matching fp16 weights with 16-byte vectors,
+// All are HBM-streaming kernels: one thread owns one 16-byte chunk of a packed row (64 weights
+// for Q2_0_g128, 80 for base-3, 128 for the binary Q1_0_g128), reads or writes the matching fp16 weights with 16-byte vectors,
 // and the grid is sized in whole waves of the SM count with a grid-stride loop.
 //
 // Ternarize rule (QAT re-ternarize step of "Metal 환경에서 ... Bonsai 8B를 파인튜닝", molayo1419.me,
@@ -68,6 +68,49 @@ __global__ void __launch_bounds__(kThreads) pack_q2_kernel(const uint16_t* __res
         const uint32_t d = out[word] ^ pw[word];
         flipped += __popc((d | (d >> 1)) & 0x55555555u);
       }
+    }
+  }
+  if (flips) {
+    flipped = __reduce_add_sync(0xFFFFFFFFu, flipped);
+    if ((threadIdx.x & 31) == 0 && flipped) atomicAdd(flips, (unsigned long long)flipped);
+  }
+}
+
+// ---- Q1_0_g128 (binary): chunk = 16 bytes = 128 weights = one group; t = -1 iff w * s < 0 ----
+__global__ void __launch_bounds__(kThreads) pack_q1_kernel(const uint16_t* __restrict__ w, int64_t w_stride,
+                                                           const uint16_t* __restrict__ s, int64_t s_stride,
+                                                           uint8_t* __restrict__ codes, int64_t c_stride,
+                                                           const uint8_t* __restrict__ prev, int64_t p_stride,
+                                                           unsigned long long* __restrict__ flips,
+                                                           int64_t n, int chunks_per_row) {
+  const int64_t total = n * chunks_per_row;
+  int flipped = 0;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i / chunks_per_row;
+    const int ch = (int)(i - row * chunks_per_row);
+    const float sv = __half2float(__ushort_as_half(s[row * s_stride + ch]));
+    const uint4* src = reinterpret_cast<const uint4*>(w + row * w_stride + (int64_t)ch * kGroup);
+    uint32_t out[4];
+#pragma unroll
+    for (int word = 0; word < 4; word++) {
+      uint32_t acc = 0;
+#pragma unroll
+      for (int v = 0; v < 4; v++) {  // 8 weights per vector, 32 per word
+        const uint4 q = __ldg(src + 4 * word + v);
+        const uint32_t pr[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int e = 0; e < 8; e++) {
+          const float wv = __half2float(__ushort_as_half((uint16_t)(pr[e / 2] >> (16 * (e & 1)))));
+          const bool neg = (wv < 0.f && sv > 0.f) || (wv > 0.f && sv < 0.f);
+          acc |= (neg ? 0u : 1u) << (8 * v + e);
+        }
+      }
+      out[word] = acc;
+    }
+    *reinterpret_cast<uint4*>(codes + row * c_stride + (int64_t)ch * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+    if (prev) {  // a weight flips when its sign bit differs from the previous packing
+      const uint4 pv = __ldg(reinterpret_cast<const uint4*>(prev + row * p_stride + (int64_t)ch * 16));
+      flipped += __popc(out[0] ^ pv.x) + __popc(out[1] ^ pv.y) + __popc(out[2] ^ pv.z) + __popc(out[3] ^ pv.w);
     }
   }
   if (flips) {
@@ -152,7 +195,7 @@ __global__ void __launch_bounds__(kThreads) unpack_kernel(const uint8_t* __restr
                                                           int8_t* __restrict__ t_out, int64_t t_stride,
                                                           int32_t* __restrict__ invalid_count,
                                                           int64_t n, int k, int chunks_per_row) {
-  constexpr int W = (LAYOUT == TERN_Q2_0_G128) ? 64 : 80;  // weights per 16-byte chunk
+  constexpr int W = (LAYOUT == TERN_Q2_0_G128) ? 64 : (LAYOUT == TERN_Q1_0_G128) ? 128 : 80;  // weights per chunk
   const int64_t total = n * chunks_per_row;
   int bad = 0;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
@@ -165,7 +208,10 @@ __global__ void __launch_bounds__(kThreads) unpack_kernel(const uint8_t* __restr
 #pragma unroll
     for (int b = 0; b < 16; b++) {
       const uint32_t byte = (qw[b / 4] >> (8 * (b % 4))) & 0xFFu;
-      if (LAYOUT == TERN_Q2_0_G128) {
+      if (LAYOUT == TERN_Q1_0_G128) {
+#pragma unroll
+        for (int f = 0; f < 8; f++) t[8 * b + f] = ((byte >> f) & 1u) ? (int8_t)1 : (int8_t)-1;
+      } else if (LAYOUT == TERN_Q2_0_G128) {
 #pragma unroll
         for (int f = 0; f < 4; f++) {
           const uint32_t c = (byte >> (2 * f)) & 3u;  // 2-bit two's complement; 0b10 is invalid
@@ -238,6 +284,9 @@ cudaError_t launch_pack(int32_t layout, int64_t n, int64_t k, const uint16_t* w,
   if (layout == TERN_Q2_0_G128)
     pack_q2_kernel<<<grid, kThreads, 0, st>>>(w, w_stride, s, s_stride, codes, c_stride, prev, p_stride, flips, n,
                                               chunks);
+  else if (layout == TERN_Q1_0_G128)
+    pack_q1_kernel<<<grid, kThreads, 0, st>>>(w, w_stride, s, s_stride, codes, c_stride, prev, p_stride, flips, n,
+                                              chunks);
   else
     pack_t3_kernel<<<grid, kThreads, 0, st>>>(w, w_stride, s, s_stride, codes, c_stride, prev, p_stride, flips, n,
                                               (int)k, chunks);
@@ -251,6 +300,10 @@ cudaError_t launch_unpack(const tern_matrix& W, uint16_t* w_out, int64_t w_strid
   const uint8_t* c = static_cast<const uint8_t*>(W.codes);
   if (W.layout == TERN_Q2_0_G128)
     unpack_kernel<TERN_Q2_0_G128><<<grid, kThreads, 0, st>>>(c, W.code_row_stride, W.scales, W.scale_row_stride,
+                                                             w_out, w_stride, t_out, t_stride, invalid_count,
+                                                             W.n, (int)W.k, chunks);
+  else if (W.layout == TERN_Q1_0_G128)
+    unpack_kernel<TERN_Q1_0_G128><<<grid, kThreads, 0, st>>>(c, W.code_row_stride, W.scales, W.scale_row_stride,
                                                              w_out, w_stride, t_out, t_stride, invalid_count,
                                                              W.n, (int)W.k, chunks);
   else

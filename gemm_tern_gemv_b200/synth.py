@@ -46,6 +46,16 @@ def ternary_codes(n: int, k: int, seed: int, p_zero: float = 0.4) -> np.ndarray:
     return out.reshape(n, k)
 
 
+def binary_codes(n: int, k: int, seed: int) -> np.ndarray:
+    """int8 [n][k] of t in {-1,+1} with P(+1) = P(-1) = 1/2 (the binary layout's codes)."""
+    return ternary_codes(n, k, seed, p_zero=0.0)
+
+
+def codes_for(layout: int, n: int, k: int, seed: int) -> np.ndarray:
+    """Codes of the distribution a layout holds: binary for layout 3 (Q1_0_g128), else ternary."""
+    return binary_codes(n, k, seed) if layout == 3 else ternary_codes(n, k, seed)
+
+
 def group_scales(n: int, groups: int, seed: int, sigma: float = 0.02) -> np.ndarray:
     """float16 [n][groups] = fp16(|N(0,1)|*sigma)."""
     rng = _rng(seed, _S_SCALES)

@@ -20,6 +20,11 @@
  *                    value 121 (five c = 1 trits). About 1.725 bits per weight at K = 5120, a
  *                    stand-in for the denser PTQ1_0 packing of the same section. A byte > 242
  *                    is invalid.
+ *   TERN_Q1_0_G128   binary sibling, t in {-1, +1} ("Bonsai 27B와 1비트가 살아남는 법", section
+ *                    "ternary와 binary가 뭔가": binary with the group scale is 1.125 bits per
+ *                    weight; the 1-bit GGUF Q1_0_g128 of that page's model card): weight k of a
+ *                    row is bit k%8 of byte k/8, 1 = +1 and 0 = -1. A row is K/8 bytes; every bit
+ *                    pattern is valid. tern_pack binarizes: t = -1 exactly when w * s < 0.
  * Scales are a separate fp16 array s[n][g], g = k / 128, with a row stride in halves.
  *
  * Conventions for every call:
@@ -70,7 +75,8 @@ typedef enum tern_status {
 
 typedef enum tern_layout {
   TERN_Q2_0_G128 = 1,
-  TERN_T3_5PB_G128 = 2
+  TERN_T3_5PB_G128 = 2,
+  TERN_Q1_0_G128 = 3
 } tern_layout;
 
 /* Bits of the device status word that tern_gemm writes (atomic OR) when it is non-NULL. */
@@ -90,7 +96,8 @@ typedef struct tern_matrix {
 
 /* ---- size arithmetic (host only, no CUDA) ------------------------------------------------ */
 
-/* Minimum packed row stride in bytes: K/4 for Q2_0_g128, ceil(K/5) rounded up to 16 for base-3.
+/* Minimum packed row stride in bytes: K/4 for Q2_0_g128, ceil(K/5) rounded up to 16 for base-3,
+ * K/8 for Q1_0_g128.
  * Returns -1 for an unknown layout or K not a positive multiple of 128. */
 TERN_API int64_t tern_row_bytes(int32_t layout, int64_t k);
 
@@ -99,7 +106,7 @@ TERN_API int64_t tern_row_bytes(int32_t layout, int64_t k);
 TERN_API int64_t tern_packed_bytes(int32_t layout, int64_t n, int64_t k);
 
 /* Stored bits per weight at the minimum stride, counting the fp16 scale per 128 weights:
- * exactly 2.125 for Q2_0_g128; 1.725 for base-3 at K = 5120 ("두 가지 패킹" section's
+ * exactly 2.125 for Q2_0_g128 and 1.125 for Q1_0_g128; 1.725 for base-3 at K = 5120 ("두 가지 패킹" section's
  * containers and the information bound log2(3) + 16/128 of section "그룹 단위 스케일을 공유하는
  * 삼진 형식", eq. b_eff, bound it from below). Returns -1 on invalid arguments. */
 TERN_API double tern_bits_per_weight(int32_t layout, int64_t k);
@@ -110,7 +117,8 @@ TERN_API double tern_bits_per_weight(int32_t layout, int64_t k);
  * paragraph "그것을 파인튜닝하는 방법": ternarize each 128-weight group on every forward pass,
  * then re-pack to 2 bits): t = round(clamp(w / s, -1, 1)) per weight with its group's scale,
  * ties |w/s| = 1/2 rounding to even (t = 0); s == 0 or NaN, or w NaN, give t = 0. The result is
- * bit-identical to that rule evaluated with exact division.
+ * bit-identical to that rule evaluated with exact division. For TERN_Q1_0_G128 the rule is the
+ * binary one: t = -1 exactly when w * s < 0, else +1 (zero, NaN and s == 0 give +1).
  *   w       device fp16 [n][w_row_stride] latent weights (first k of each row used)
  *   scales  device fp16 [n][scale_row_stride]
  *   codes   device uint8 [n][code_row_stride] output; exactly tern_row_bytes(layout, k) bytes of
@@ -128,7 +136,7 @@ TERN_API tern_status tern_pack(int32_t layout, int64_t n, int64_t k,
  *   prev_codes       device uint8 [n][prev_row_stride]: the previous packed codes, same layout and
  *                    k; must not overlap `codes`
  *   flips            device uint64: the number of weights (k < K) whose code field (Q2 2-bit field,
- *                    base-3 digit) differs from prev_codes is ADDED (the caller zeroes it); for
+ *                    base-3 digit, binary sign bit) differs from prev_codes is ADDED (the caller zeroes it); for
  *                    valid codes that is the number of weights whose t changed
  * Errors: those of tern_pack; TERN_ERR_INVALID_ARG for NULL prev_codes / flips, prev_codes ==
  *         codes or a short prev_row_stride; TERN_ERR_ALIGNMENT for a misaligned prev_codes,
@@ -159,15 +167,17 @@ TERN_API size_t tern_gemv_workspace_bytes(const tern_matrix* W, int64_t batch);
 /* y[b][n] = sum_g s[n][g] * sum_{k in group g} t[n][k] * x[b][k] for b < batch; fp32
  * accumulation, fp16 result. Small batches run on mma.sync kernels that decode the codes in
  * registers; batches of 17 or more with n % 8 == 0 run on the tcgen05 kernel of tern_gemm (no
- * workspace). The result of a call depends only on (W, x, batch) and the device.
+ * workspace). A Q1_0_g128 batch below that runs as one register-kernel launch per two rows of x.
+ * The result of a call depends only on (W, x, batch) and the device.
  *   x          device fp16 [batch][k], contiguous
  *   y          device fp16 [batch][n], contiguous
  *   workspace  device, >= tern_gemv_workspace_bytes(W, batch) bytes, 16-byte aligned; may be
  *              NULL when that size is 0. Its trailing counter words must be zero before the first
  *              call that uses this workspace (e.g. cudaMemset once); every call leaves them zero
  *              again. Calls that share a workspace must not overlap on the GPU.
- * Errors: TERN_ERR_INVALID_ARG (batch outside 1..64, ...), TERN_ERR_UNSUPPORTED,
- *         TERN_ERR_ALIGNMENT, TERN_ERR_WORKSPACE, TERN_ERR_CUDA. */
+ * Errors: TERN_ERR_INVALID_ARG (batch outside 1..64, ...), TERN_ERR_UNSUPPORTED (also a Q1_0_g128
+ *         matrix of 2^30 or more (32-row tile, 512-weight window) units at a batch the GEMM kernel
+ *         does not take), TERN_ERR_ALIGNMENT, TERN_ERR_WORKSPACE, TERN_ERR_CUDA. */
 TERN_API tern_status tern_gemv(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y,
                       void* workspace, size_t workspace_bytes, void* stream);
 
@@ -206,8 +216,9 @@ TERN_API tern_status tern_gemv_noalloc(const tern_matrix* W, const uint16_t* x, 
  *   device_status  device uint32 or NULL: TERN_DEVICE_TIMEOUT is OR-ed in if an internal pipeline
  *                  wait exceeds its bound (the kernel then abandons its work and exits; Y is
  *                  incomplete). The caller zeroes it.
- * Both layouts: a base-3 K block of 64 weights spans at most 14 bytes and is decoded through a
- * byte -> five-field table; Q2_0_g128 through one masked multiply per pair of weights.
+ * Every layout: a base-3 K block of 64 weights spans at most 14 bytes and is decoded through a
+ * byte -> five-field table; Q2_0_g128 and Q1_0_g128 through one masked multiply per pair of
+ * weights.
  * Errors: TERN_ERR_INVALID_ARG, TERN_ERR_UNSUPPORTED (unknown layout), TERN_ERR_ALIGNMENT,
  * TERN_ERR_CUDA. */
 TERN_API tern_status tern_gemm(const tern_matrix* W, const uint16_t* X, int64_t m, uint16_t* Y,

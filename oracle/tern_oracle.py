@@ -31,6 +31,11 @@ Readings of points the pages leave open (each is stated where it is used):
       (five c = 1 trits) up to a multiple of 16 bytes.
   R3  Ternarize: t = round(clamp(w/s, -1, 1)) with w/s exact (fp64 quotient of two fp16 values)
       and round-half-to-even, so exact ties |w/s| = 1/2 give 0; s == 0, s NaN or w NaN give 0.
+  R12 Binary layout (Q1_0_g128, weights in {-1, +1}, one fp16 scale per 128; [velog-27B] section
+      "ternary와 binary가 뭔가": binary 1.125 bits per weight; [Metal-8B] opening paragraph "이
+      모델들이란 무엇인가": binary weights share one fp16 scale per 128): weight k of a row is bit
+      k % 8 of byte k / 8, 1 = +1 and 0 = -1; every bit pattern is valid; rows are K/8 bytes
+      (a multiple of 16). Binarize: t = -1 exactly when w * s < 0 (zero and NaN give +1).
   R4  Products take x as given (any rotation of x is the caller's step) and are compared with
       |y - y_ref| <= 2e-3 * sum_k |w_k x_k| + 1e-5.
 """
@@ -43,7 +48,8 @@ import numpy as np
 GROUP = 128
 Q2_0_G128 = 1
 T3_5PB_G128 = 2
-LAYOUTS = (Q2_0_G128, T3_5PB_G128)
+Q1_0_G128 = 3
+LAYOUTS = (Q2_0_G128, T3_5PB_G128, Q1_0_G128)
 
 T3_PAD_BYTE = 121  # 1 + 3 + 9 + 27 + 81: five trits with c = 1 (t = 0)
 _POW3 = (1, 3, 9, 27, 81)
@@ -69,6 +75,8 @@ def _check(layout: int, k: int) -> None:
 def code_bytes(layout: int, k: int) -> int:
     """Bytes that carry the K codes of one row, before the 16-byte row padding (R1, R2)."""
     _check(layout, k)
+    if layout == Q1_0_G128:
+        return k // 8  # R12: one bit per weight
     return k // 4 if layout == Q2_0_G128 else -(-k // 5)
 
 
@@ -102,7 +110,12 @@ def pack(t: np.ndarray, layout: int) -> np.ndarray:
     if t.size and (t.min() < -1 or t.max() > 1):
         raise ValueError("codes must be in {-1, 0, +1}")
     out = np.zeros((n, row_bytes(layout, k)), dtype=np.uint8)
-    if layout == Q2_0_G128:
+    if layout == Q1_0_G128:
+        if t.size and (t == 0).any():
+            raise ValueError("binary codes must be in {-1, +1}")
+        bit = (t > 0).astype(np.int64).reshape(n, k // 8, 8)  # R12: bit k % 8 of byte k / 8
+        out[:, : k // 8] = sum(bit[:, :, i] << i for i in range(8)).astype(np.uint8)
+    elif layout == Q2_0_G128:
         c = t.astype(np.int64) & 3  # R1: 2-bit two's complement
         c4 = c.reshape(n, k // 4, 4)
         byte = c4[:, :, 0] + (c4[:, :, 1] << 2) + (c4[:, :, 2] << 4) + (c4[:, :, 3] << 6)
@@ -130,7 +143,11 @@ def unpack(codes: np.ndarray, layout: int, k: int, rows=None, check: bool = True
         codes = codes[np.asarray(rows)]
     n = codes.shape[0]
     kk = np.arange(k)
-    if layout == Q2_0_G128:
+    if layout == Q1_0_G128:
+        bit = (codes[:, kk // 8].astype(np.int64) >> (kk % 8)) & 1
+        bad = np.zeros(bit.shape, dtype=bool)
+        t = 2 * bit - 1
+    elif layout == Q2_0_G128:
         byte = codes[:, kk // 4].astype(np.int64)
         f = (byte >> (2 * (kk % 4))) & 3
         bad = f == 2
@@ -153,10 +170,21 @@ def count_invalid(codes: np.ndarray, layout: int, n: int, k: int) -> int:
     """Number of weights (row, k < K) whose code is invalid."""
     codes = np.asarray(codes, dtype=np.uint8)[:n]
     kk = np.arange(k)
+    if layout == Q1_0_G128:
+        return 0  # every bit is a valid code
     if layout == Q2_0_G128:
         f = (codes[:, kk // 4].astype(np.int64) >> (2 * (kk % 4))) & 3
         return int((f == 2).sum())
     return int((codes[:, kk // 5] > 242).sum())
+
+
+def binarize(w: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """R12: t = -1 where w * s < 0 (w and its group's scale of strictly opposite signs), else +1."""
+    w = np.asarray(w, dtype=np.float16).astype(np.float64)
+    n, k = w.shape
+    s = np.repeat(np.asarray(scales, dtype=np.float16)[:, : k // GROUP].astype(np.float64), GROUP, axis=1)
+    neg = ((w < 0) & (s > 0)) | ((w > 0) & (s < 0))
+    return np.where(neg, -1, 1).astype(np.int8)
 
 
 def count_flips(old_codes: np.ndarray, new_codes: np.ndarray, layout: int, k: int) -> int:
@@ -167,7 +195,10 @@ def count_flips(old_codes: np.ndarray, new_codes: np.ndarray, layout: int, k: in
     new = np.asarray(new_codes, dtype=np.uint8)
     _check(layout, k)
     kk = np.arange(k)
-    if layout == Q2_0_G128:
+    if layout == Q1_0_G128:
+        f_old = (old[:, kk // 8] >> (kk % 8)) & 1
+        f_new = (new[:, kk // 8] >> (kk % 8)) & 1
+    elif layout == Q2_0_G128:
         f_old = (old[:, kk // 4] >> (2 * (kk % 4))) & 3
         f_new = (new[:, kk // 4] >> (2 * (kk % 4))) & 3
     else:

@@ -29,7 +29,10 @@ def ternarize_rows(w: np.ndarray, s: np.ndarray) -> np.ndarray:
 
 def workload(layout: int, n: int, k: int, batch: int, seed: int, p_zero: float = 0.4):
     """(codes uint8 [n][row_bytes], scales fp16 [n][k/128], x fp16 [batch][k])."""
-    t = synth.ternary_codes(n, k, seed, p_zero=p_zero)
+    if layout == O.Q1_0_G128:
+        t = synth.binary_codes(n, k, seed)
+    else:
+        t = synth.ternary_codes(n, k, seed, p_zero=p_zero)
     s = synth.group_scales(n, k // 128, seed)
     x = synth.activations(batch, k, seed)
     return pack_rows(t, layout), s, x

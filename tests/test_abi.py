@@ -46,14 +46,16 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_size_arithmetic_matches_oracle(lib):
-    for layout in (T.Q2_0_G128, T.T3_5PB_G128):
+    for layout in (T.Q2_0_G128, T.T3_5PB_G128, T.Q1_0_G128):
         for k in list(range(128, 20000, 128)) + [151936 // 128 * 128]:
             assert T.row_bytes(layout, k) == O.row_bytes(layout, k)
             assert T.packed_bytes(layout, 7, k) == O.packed_bytes(layout, 7, k)
             assert T.bits_per_weight(layout, k) == pytest.approx(O.bits_per_weight(layout, k), abs=0, rel=1e-15)
     assert T.bits_per_weight(T.Q2_0_G128, 4096) == 2.125
     assert T.bits_per_weight(T.T3_5PB_G128, 5120) == 1.725
-    assert lib.tern_row_bytes(3, 128) == -1
+    assert T.bits_per_weight(T.Q1_0_G128, 4096) == 1.125
+    assert lib.tern_row_bytes(4, 128) == -1
+    assert lib.tern_row_bytes(0, 128) == -1
     assert lib.tern_row_bytes(1, 100) == -1
     assert lib.tern_row_bytes(1, 0) == -1
     assert lib.tern_packed_bytes(1, 0, 128) == -1
@@ -79,7 +81,7 @@ def _mat(**kw):
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(layout=0), 2), (dict(layout=3), 2), (dict(n=0), 1), (dict(k=1000), 1), (dict(k=0), 1),
+    (dict(layout=0), 2), (dict(layout=4), 2), (dict(n=0), 1), (dict(k=1000), 1), (dict(k=0), 1),
     (dict(codes=0), 1), (dict(scales=0), 1), (dict(code_row_stride=128), 1), (dict(scale_row_stride=4), 1),
     (dict(codes=FAKE + 8), 3), (dict(scales=FAKE + 2), 3), (dict(code_row_stride=264), 3),
     (dict(scale_row_stride=12), 3),
@@ -120,9 +122,21 @@ def test_gemv_workspace_size_and_rejection(lib):
     assert lib.tern_gemv_workspace_bytes(None, 1) == 0
 
 
+def test_binary_gemv_workspace_is_that_of_two_rows(lib):
+    # the binary register kernel runs batch rows in pairs, one launch after another on the stream,
+    # so every batch below the GEMM's reuses the workspace of a two-row launch
+    m = _mat(layout=3, n=4096, k=4096, code_row_stride=512, scale_row_stride=32)
+    two = lib.tern_gemv_workspace_bytes(ctypes.byref(m), 2)
+    assert two > 0
+    for b in (3, 7, 16):
+        assert lib.tern_gemv_workspace_bytes(ctypes.byref(m), b) == two
+    assert lib.tern_gemv_workspace_bytes(ctypes.byref(m), 17) == 0  # the GEMM kernel takes it
+
+
 def test_pack_unpack_gemm_reject(lib):
     P = lambda v: ctypes.c_void_p(v)
-    assert lib.tern_pack(3, 4, 128, P(FAKE), 128, P(FAKE), 8, P(FAKE), 32, None) == 2
+    assert lib.tern_pack(4, 4, 128, P(FAKE), 128, P(FAKE), 8, P(FAKE), 32, None) == 2
+    assert lib.tern_pack(3, 4, 256, P(FAKE), 256, P(FAKE), 8, P(FAKE), 16, None) == 1  # binary row needs 32
     assert lib.tern_pack(1, 4, 130, P(FAKE), 136, P(FAKE), 8, P(FAKE), 48, None) == 1
     assert lib.tern_pack(1, 4, 128, P(FAKE), 120, P(FAKE), 8, P(FAKE), 32, None) == 1
     assert lib.tern_pack(1, 4, 128, P(FAKE + 4), 128, P(FAKE), 8, P(FAKE), 32, None) == 3
@@ -133,7 +147,9 @@ def test_pack_unpack_gemm_reject(lib):
     assert lib.tern_unpack(ctypes.byref(m), P(FAKE), 1028, None, 0, None, None) == 3
     t3 = _mat(layout=2, code_row_stride=208)
     assert lib.tern_gemm(ctypes.byref(t3), P(FAKE), 0, P(FAKE), None, None) == 1  # base-3 accepted up to m
-    assert lib.tern_gemm(ctypes.byref(_mat(layout=3)), P(FAKE), 16, P(FAKE), None, None) == 2
+    q1 = _mat(layout=3, code_row_stride=128)
+    assert lib.tern_gemm(ctypes.byref(q1), P(FAKE), 0, P(FAKE), None, None) == 1  # binary accepted up to m
+    assert lib.tern_gemm(ctypes.byref(_mat(layout=4)), P(FAKE), 16, P(FAKE), None, None) == 2
     assert lib.tern_gemm(ctypes.byref(m), P(FAKE), 0, P(FAKE), None, None) == 1
     assert lib.tern_gemm(ctypes.byref(_mat(n=60)), P(FAKE), 16, P(FAKE), None, None) == 3
 

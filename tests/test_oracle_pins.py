@@ -68,10 +68,11 @@ def test_row_bytes_closed_forms():
         assert O.row_bytes(O.Q2_0_G128, k) == k // 4
         rb = O.row_bytes(O.T3_5PB_G128, k)
         assert rb % 16 == 0 and rb * 5 >= k and (rb - 16) * 5 < k
+        assert O.row_bytes(O.Q1_0_G128, k) == k // 8
     with pytest.raises(ValueError):
         O.row_bytes(O.Q2_0_G128, 100)
     with pytest.raises(ValueError):
-        O.row_bytes(3, 128)
+        O.row_bytes(4, 128)
 
 
 # ---------------------------------------------------------------- exhaustive byte tables
@@ -134,7 +135,7 @@ def test_t3_padding_bytes():
 @pytest.mark.parametrize("layout", O.LAYOUTS)
 @pytest.mark.parametrize("k", [128, 256, 384, 640, 1024, 1152, 4096, 5120])
 def test_round_trip(layout, k):
-    t = synth.ternary_codes(17, k, seed=k + layout)
+    t = synth.codes_for(layout, 17, k, seed=k + layout)
     p = O.pack(t, layout)
     assert p.shape == (17, O.row_bytes(layout, k))
     assert np.array_equal(O.unpack(p, layout, k), t)
@@ -216,7 +217,7 @@ def _brute(t, s, x):
 def test_gemv_integer_bruteforce(layout):
     rng = np.random.default_rng(1)
     for n, k, b in ((1, 128, 1), (7, 256, 3), (33, 384, 2), (5, 640, 9)):
-        t = synth.ternary_codes(n, k, seed=n * k)
+        t = synth.codes_for(layout, n, k, seed=n * k)
         s = np.ones((n, k // 128), dtype=np.float16)
         x = rng.integers(-2, 3, size=(b, k)).astype(np.float16)
         y, a = O.gemv(O.pack(t, layout), s, x, layout, k)
@@ -228,7 +229,7 @@ def test_gemv_integer_bruteforce(layout):
 @pytest.mark.parametrize("layout", O.LAYOUTS)
 def test_gemv_exact_rational(layout):
     n, k, b = 6, 384, 2
-    t = synth.ternary_codes(n, k, seed=21)
+    t = synth.codes_for(layout, n, k, seed=21)
     s = synth.group_scales(n, k // 128, seed=21)
     x = synth.activations(b, k, seed=21)
     y, a = O.gemv(O.pack(t, layout), s, x, layout, k)
@@ -360,10 +361,10 @@ def test_planted_mistakes_are_caught():
     assert not np.allclose(_gemv_scale_wrong_group(p, sc, x, O.Q2_0_G128, k), ex, rtol=1e-3)
 
 
-@pytest.mark.parametrize("layout", [O.Q2_0_G128, O.T3_5PB_G128])
+@pytest.mark.parametrize("layout", O.LAYOUTS)
 def test_count_flips_pins(layout):
     k = 640
-    t1 = synth.ternary_codes(40, k, seed=11)
+    t1 = synth.codes_for(layout, 40, k, seed=11)
     p1 = O.pack(t1, layout)
     assert O.count_flips(p1, p1, layout, k) == 0
     # any set of changed weights: the count is the number of changed t (unpack is an independent read)
@@ -371,7 +372,7 @@ def test_count_flips_pins(layout):
     rng = np.random.default_rng(12)
     for _ in range(37):
         r, c = rng.integers(0, 40), rng.integers(0, k)
-        t2[r, c] = (t2[r, c] + 2) % 3 - 1  # -1 -> 0 -> 1 -> -1
+        t2[r, c] = -t2[r, c] if layout == O.Q1_0_G128 else (t2[r, c] + 2) % 3 - 1  # -1 -> 0 -> 1 -> -1
     p2 = O.pack(t2, layout)
     assert O.count_flips(p1, p2, layout, k) == int((O.unpack(p1, layout, k) != O.unpack(p2, layout, k)).sum())
     assert O.count_flips(p1, p2, layout, k) == int((t1 != t2).sum())
@@ -408,3 +409,56 @@ def test_transposed_product_is_the_adjoint(layout):
     ones = np.ones((n, k // 128), dtype=np.float16)
     dxi, _ = O.gemv_t(codes, ones, dy, layout, k)
     assert np.array_equal(dxi, dy.astype(np.int64) @ t.astype(np.int64))
+
+
+
+# ---------------------------------------------------------------- binary layout (R12)
+def test_q1_bits_per_weight_is_the_pages_figure():
+    # [velog-27B] "ternary와 binary가 뭔가": binary with a group scale is 1.125 bits per weight
+    for k in (128, 1024, 4096, 5120, 17408):
+        assert O.bits_per_weight(O.Q1_0_G128, k) == 1.125
+
+
+def test_q1_byte_table_exhaustive():
+    # every byte value is valid and its 8 weights are its bits, LSB first, 1 -> +1, 0 -> -1
+    codes = np.arange(256, dtype=np.uint8).reshape(256, 1).repeat(16, axis=1)
+    t = O.unpack(codes, O.Q1_0_G128, 128)
+    for v in range(256):
+        want = [1 if (v >> i) & 1 else -1 for i in range(8)]
+        assert t[v, :8].tolist() == want
+    assert O.count_invalid(codes, O.Q1_0_G128, 256, 128) == 0
+    assert np.array_equal(O.pack(t, O.Q1_0_G128), codes)
+
+
+def test_q1_hand_packed():
+    t = np.full((1, 128), -1, dtype=np.int8)
+    t[0, [0, 3, 9, 127]] = 1
+    p = O.pack(t, O.Q1_0_G128)
+    assert p[0, 0] == 0b00001001 and p[0, 1] == 0b00000010 and p[0, 15] == 0x80 and p[0, 2:15].sum() == 0
+    with pytest.raises(ValueError):
+        O.pack(np.zeros((1, 128), dtype=np.int8), O.Q1_0_G128)  # 0 is not a binary code
+
+
+def test_binarize_rule():
+    s = np.array([[1.0], [-2.0], [0.0]], dtype=np.float16)
+    w = np.array([[0.5, -0.5, 0.0, np.nan] + [1.0] * 124,
+                  [0.5, -0.5, 0.0, np.nan] + [1.0] * 124,
+                  [0.5, -0.5, 0.0, np.nan] + [1.0] * 124], dtype=np.float16)
+    t = O.binarize(w, s)
+    assert t[0, :4].tolist() == [1, -1, 1, 1]
+    assert t[1, :4].tolist() == [-1, 1, 1, 1]
+    assert t[2, :4].tolist() == [1, 1, 1, 1]
+    # binarizing s * t reproduces t (lossless re-encode, [Metal-8B])
+    tt = np.where(synth.ternary_codes(8, 256, seed=3) >= 0, 1, -1).astype(np.int8)
+    sc = synth.group_scales(8, 2, seed=3)
+    assert np.array_equal(O.binarize(O.dequantize(tt, sc).astype(np.float16), sc), tt)
+
+
+def test_q1_gemv_integer_bruteforce():
+    rng = np.random.default_rng(41)
+    t = np.where(rng.random((9, 256)) < 0.5, -1, 1).astype(np.int8)
+    x = rng.integers(-3, 4, size=(2, 256)).astype(np.float16)
+    ones = np.ones((9, 2), dtype=np.float16)
+    y, a = O.gemv(O.pack(t, O.Q1_0_G128), ones, x, O.Q1_0_G128, 256)
+    want = np.array([[sum(int(t[r, c]) * int(x[b, c]) for c in range(256)) for r in range(9)] for b in range(2)])
+    assert np.array_equal(y, want)

@@ -27,7 +27,7 @@ def _noalloc(W, x, y):
                                      ctypes.c_void_p(y.data_ptr()), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
-@pytest.mark.parametrize("layout", [T.Q2_0_G128, T.T3_5PB_G128])
+@pytest.mark.parametrize("layout", [T.Q2_0_G128, T.T3_5PB_G128, T.Q1_0_G128])
 @pytest.mark.parametrize("n,k,batch", [(4096, 4096, 1), (5120, 17408, 1), (1000, 2176, 3), (4096, 12288, 8),
                                        (24576, 4096, 1), (300, 640, 2)])
 def test_noalloc_matches_gemv_twice(layout, n, k, batch):
