@@ -98,27 +98,67 @@ def profiled_traffic(kernel_key: str):
 
 
 class ClockSampler:
-    """Samples nvidia-smi SM clock / throttle reasons every 200 ms; only the samples taken between
-    begin() and end() (the timed region) enter the summary."""
+    """Samples the SM clock, power and clock-event (throttle) reasons of one GPU while the timed region
+    runs; only samples taken between begin() and end() enter the summary. NVML is polled every 2 ms
+    from a thread (so even a short region gets samples); without NVML, `nvidia-smi -lms 200` is read."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, pci_bus_id: str | None = None):
         self.index = index
-        self.rows = []  # (host time, fields)
+        self.pci = pci_bus_id
+        self.rows = []  # (host time, sm MHz, max sm MHz, power W, reason names)
         self.proc = None
         self.thread = None
+        self.stop = threading.Event()
+        self.source = None
         self.t0 = self.t1 = None
 
     def __enter__(self):
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            h = None
+            if self.pci:
+                try:
+                    h = nv.nvmlDeviceGetHandleByPciBusId(self.pci)
+                except Exception:
+                    h = None
+            if h is None:
+                h = nv.nvmlDeviceGetHandleByIndex(self.index)
+            bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown | nv.nvmlClocksEventReasonHwPowerBrakeSlowdown,
+                    "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+            mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+
+            def poll():
+                while not self.stop.is_set():
+                    try:
+                        sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                        pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                        r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.rows.append((time.time(), sm, mx, pw, [k for k, b in bits.items() if r & b]))
+                    except Exception:
+                        pass
+                    time.sleep(0.002)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            self.source = "nvml, 2 ms polling"
+            return self
+        except Exception:
+            pass
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "200"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            self.source = "nvidia-smi -lms 200"
             deadline = time.time() + 5.0  # nvidia-smi takes a moment to print its first sample
             while not self.rows and time.time() < deadline and self.proc.poll() is None:
                 time.sleep(0.02)
@@ -127,10 +167,16 @@ class ClockSampler:
         return self
 
     def _read(self):
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
         for line in self.proc.stdout:
             parts = [x.strip() for x in line.split(",")]
             if len(parts) >= 9:
-                self.rows.append((time.time(), parts))
+                names = [self.NAMES[i] for i in range(4) if parts[5 + i].lower() == "active"]
+                self.rows.append((time.time(), num(parts[1]), num(parts[2]), num(parts[3]), names))
 
     def begin(self):
         self.t0 = time.time()
@@ -139,6 +185,7 @@ class ClockSampler:
         self.t1 = time.time()
 
     def __exit__(self, *exc):
+        self.stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -149,17 +196,17 @@ class ClockSampler:
             self.thread.join(timeout=2)
 
     def summary(self):
-        rows = [r for (t, r) in self.rows
-                if self.t0 is not None and self.t1 is not None and self.t0 <= t <= self.t1]
+        rows = [r for r in list(self.rows)
+                if self.t0 is not None and self.t1 is not None and self.t0 <= r[0] <= self.t1]
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source}
+        sm = [r[1] for r in rows if r[1] is not None]
+        mx = [r[2] for r in rows if r[2] is not None]
+        pw = [r[3] for r in rows if r[3] is not None]
+        reasons = sorted({n for r in rows for n in r[4]})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows), "power_w_median": statistics.median(pw) if pw else None}
+                "reasons": reasons, "samples": len(rows), "power_w_median": statistics.median(pw) if pw else None,
+                "source": self.source}
 
 
 # ----------------------------------------------------------------------------- the native arm
@@ -205,7 +252,7 @@ def run_native(args, rank, world, local_rank):
 
     def step(c):
         for i in range(len(mats)):
-            T.gemv(W[c][i], xs[i], y=ys[i], workspace=wss[c][i])
+            T.gemv(W[c][i], xs[i], y=ys[i], workspace=wss[c][i], static_weights=True)
 
     # one CUDA graph per weight copy holds the six launches of a step
     graphs = []
@@ -231,7 +278,10 @@ def run_native(args, rank, world, local_rank):
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local_rank) as clk:
+    pci = None
+    if hasattr(props, "pci_bus_id"):
+        pci = f"{getattr(props, 'pci_domain_id', 0):08X}:{props.pci_bus_id:02X}:{getattr(props, 'pci_device_id', 0):02X}.0"
+    with ClockSampler(local_rank, pci) as clk:
         clk.begin()
         with torch.cuda.stream(stream):
             e0.record(stream)
@@ -270,7 +320,9 @@ def run_native(args, rank, world, local_rank):
                            "gemvs_per_step": launches_per_step, "bytes_per_step": set_bytes,
                            "l2": f"rotating {copies} weight copies ({copies * weight_bytes / 1e6:.0f} MB > 3x L2 "
                                  f"{l2 / 1e6:.0f} MB)", "parallelism": f"replicas x{world}",
-                           "hbm_frac_of_8TBps": round(value / world / 8000.0, 4)},
+                           "hbm_frac_of_8TBps": round(value / world / 8000.0, 4),
+                           "launch": "tern_gemv_ex with TERN_GEMV_STATIC_WEIGHTS (programmatic dependent launch: "
+                                     "each GEMV starts streaming its weights while the previous one finishes)"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary()}
         if extras:
@@ -296,7 +348,7 @@ def time_kernels(torch, T, W, xs, ys, wss, mats, copies, stream, reps=40):
             with torch.cuda.graph(g, stream=stream):
                 for r in range(reps):
                     c = r % copies
-                    T.gemv(W[c][i], xs[i], y=ys[i], workspace=wss[c][i])
+                    T.gemv(W[c][i], xs[i], y=ys[i], workspace=wss[c][i], static_weights=True)
             g.replay()
             torch.cuda.synchronize()
             a = torch.cuda.Event(enable_timing=True)
@@ -326,7 +378,7 @@ def measure_e2e(torch, T, W, mats, copies, args, stream, world, dev, set_bytes):
     def one(c):
         for i in range(len(mats)):
             dx[i].copy_(hx[i], non_blocking=True)
-            T.gemv(W[c][i], dx[i], y=dy[i], workspace=wss[c][i])
+            T.gemv(W[c][i], dx[i], y=dy[i], workspace=wss[c][i], static_weights=True)
             hy[i].copy_(dy[i], non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -345,7 +397,7 @@ def measure_e2e(torch, T, W, mats, copies, args, stream, world, dev, set_bytes):
     d2h = sum(t.numel() * 2 for t in hy)
     return {"value": round(set_bytes * steps * world / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "ms_per_step": round(ms / steps, 6), "path": "python binding -> tern_gemv C ABI, eager launches"}
+            "ms_per_step": round(ms / steps, 6), "path": "python binding -> tern_gemv_ex C ABI (TERN_GEMV_STATIC_WEIGHTS), eager launches"}
 
 
 def measure_extras(torch, T, dev, peaks, stream):
@@ -417,7 +469,7 @@ def measure_extras(torch, T, dev, peaks, stream):
         def f():
             c = it[0] % len(Ws)
             it[0] += 1
-            T.gemv(Ws[c], x, y=y, workspace=wss[c])
+            T.gemv(Ws[c], x, y=y, workspace=wss[c], static_weights=True)
         ms = timed(f, 20)
         nb = algorithmic_bytes(layout, n, k, b)
         flops = 2.0 * n * k * b
@@ -568,7 +620,7 @@ def run_profile_case(case: str, launches: int = 6):
         W = make_weights(torch, T, n, k, layout, 1, dev)
         x = torch.randn((b, k), device=dev).to(torch.float16)
         ws = T.gemv_workspace(W, b)
-        fn = lambda: T.gemv(W, x, workspace=ws)
+        fn = lambda: T.gemv(W, x, workspace=ws, static_weights=True)
     elif kind == "gemm":
         m, n, k = (int(v) for v in parts[2].split("x"))
         W = make_weights(torch, T, n, k, layout, 1, dev)

@@ -19,6 +19,7 @@ T3_5PB_G128 = 2
 Q1_0_G128 = 3
 GROUP = 128
 GEMV_MAX_BATCH = 64
+GEMV_STATIC_WEIGHTS = 1
 DEVICE_TIMEOUT = 1
 
 STATUS = {0: "TERN_OK", 1: "TERN_ERR_INVALID_ARG", 2: "TERN_ERR_UNSUPPORTED", 3: "TERN_ERR_ALIGNMENT",
@@ -54,6 +55,8 @@ SIGNATURES = {
     "tern_gemv_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(TernMatrixC), ctypes.c_int64]),
     "tern_gemv": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                  ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "tern_gemv_ex": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                    ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint32, ctypes.c_void_p]),
     "tern_gemv_noalloc": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                          ctypes.c_void_p]),
     "tern_gemm": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
@@ -238,8 +241,9 @@ def gemv_workspace(W: TernMatrix, batch: int):
     return torch.zeros(nb, dtype=torch.uint8, device=W.codes.device) if nb else None
 
 
-def gemv(W: TernMatrix, x, y=None, workspace=None):
-    """y [batch][n] = x [batch][k] @ W^T with W ternary (tern_gemv)."""
+def gemv(W: TernMatrix, x, y=None, workspace=None, static_weights: bool = False):
+    """y [batch][n] = x [batch][k] @ W^T with W ternary (tern_gemv; tern_gemv_ex with
+    TERN_GEMV_STATIC_WEIGHTS when `static_weights`: no pending GPU work writes W)."""
     torch = _torch()
     if x.dim() == 1:
         x = x.unsqueeze(0)
@@ -251,8 +255,13 @@ def gemv(W: TernMatrix, x, y=None, workspace=None):
         workspace = gemv_workspace(W, batch)
     wsb = workspace.numel() if workspace is not None else 0
     c = W.c()
-    st = lib().tern_gemv(ctypes.byref(c), _ptr(x), batch, _ptr(y), _ptr(workspace), wsb, _stream_handle())
-    _check(st, "tern_gemv")
+    if static_weights:
+        st = lib().tern_gemv_ex(ctypes.byref(c), _ptr(x), batch, _ptr(y), _ptr(workspace), wsb,
+                                GEMV_STATIC_WEIGHTS, _stream_handle())
+        _check(st, "tern_gemv_ex")
+    else:
+        st = lib().tern_gemv(ctypes.byref(c), _ptr(x), batch, _ptr(y), _ptr(workspace), wsb, _stream_handle())
+        _check(st, "tern_gemv")
     return y
 
 

@@ -136,6 +136,12 @@ size_t tern_gemv_workspace_bytes(const tern_matrix* W, int64_t batch) {
 
 tern_status tern_gemv(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y,
                       void* workspace, size_t workspace_bytes, void* stream) {
+  return tern_gemv_ex(W, x, batch, y, workspace, workspace_bytes, 0u, stream);
+}
+
+tern_status tern_gemv_ex(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y, void* workspace,
+                         size_t workspace_bytes, uint32_t flags, void* stream) {
+  if (flags & ~(uint32_t)TERN_GEMV_STATIC_WEIGHTS) return TERN_ERR_INVALID_ARG;
   tern_status s = check_matrix(W);
   if (s != TERN_OK) return s;
   if (batch < 1 || batch > TERN_GEMV_MAX_BATCH || !x || !y) return TERN_ERR_INVALID_ARG;
@@ -146,7 +152,7 @@ tern_status tern_gemv(const tern_matrix* W, const uint16_t* x, int64_t batch, ui
     if (!workspace || workspace_bytes < plan.ws_bytes) return TERN_ERR_WORKSPACE;
     if (!aligned16(workspace)) return TERN_ERR_ALIGNMENT;
   }
-  return from_cuda(launch_gemv(*W, x, (int)batch, y, workspace, plan, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_gemv(*W, x, (int)batch, y, workspace, plan, static_cast<cudaStream_t>(stream), flags));
 }
 
 tern_status tern_gemv_noalloc(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y, void* stream) {

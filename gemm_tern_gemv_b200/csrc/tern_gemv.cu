@@ -61,6 +61,7 @@ struct Args {
   int run;          // register kernel: (tile, window) units per warp run (stream-K)
   int kmax;         // register kernel: partial-sum slots per tile and slice
   uint32_t unit;    // always 1 (see `mul` in the kernel)
+  int early;        // register kernel: W may be read before earlier work on the stream completes
 };
 
 // ---- small device helpers --------------------------------------------------------------------
@@ -888,6 +889,9 @@ __global__ void __launch_bounds__(kSThreads, kRegCtasPerSm)
   }
   if (threadIdx.x == 0) *abort_flag = 0;
   __syncwarp();
+  // The next kernel on the stream may be scheduled as soon as this grid's CTAs leave their SMs
+  // (programmatic dependent launch; a no-op for plain launches).
+  sm100::griddep_launch_dependents();
 
   // this warp's run of (tile, window) units in the slice (empty past the last run); runs are dealt
   // to CTAs round-robin so both CTAs on an SM, and all SMs, get the same number of runs (+-1)
@@ -919,7 +923,13 @@ __global__ void __launch_bounds__(kSThreads, kRegCtasPerSm)
       ++is_tile;
     }
   };
-  if (lane == 0)
+  // With a.early the first code / scale boxes are requested before waiting for the preceding grid: the
+  // caller guarantees that no work still in flight writes W. x, y and the workspace are only touched
+  // after the wait, which returns at once for plain launches.
+  if (a.early && lane == 0)
+    for (int st = 0; st < STAGES && st < total; st++) issue_next();
+  sm100::griddep_wait();
+  if (!a.early && lane == 0)
     for (int st = 0; st < STAGES && st < total; st++) issue_next();
 
   s_build_frag<LAYOUT, BS>(a, g0, ngroups, nwin_alloc, frag);
@@ -1171,8 +1181,23 @@ cudaError_t launch_reg(const CUtensorMap& tc, const CUtensorMap& ts, const Args&
   auto kern = gemv_reg_kernel<LAYOUT, RT, BS, STAGES>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(grid_x, a.splits), kSThreads, smem, st>>>(tc, ts, a);
-  return cudaGetLastError();
+  if (!a.early) {
+    kern<<<dim3(grid_x, a.splits), kSThreads, smem, st>>>(tc, ts, a);
+    return cudaGetLastError();
+  }
+  // programmatic dependent launch: the grid may start while the preceding kernel finishes
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid_x, a.splits);
+  cfg.blockDim = dim3(kSThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tc, ts, a);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 #ifndef TERN_REG_RT
@@ -1312,7 +1337,7 @@ GemvPlan gemv_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms)
 }
 
 cudaError_t launch_gemv(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y, void* workspace,
-                        const GemvPlan& plan, cudaStream_t st) {
+                        const GemvPlan& plan, cudaStream_t st, uint32_t flags) {
   if (plan.gemm) return launch_gemm(W, x, batch, y, nullptr, st);
   Args a;
   a.codes = static_cast<const uint8_t*>(W.codes);
@@ -1331,6 +1356,7 @@ cudaError_t launch_gemv(const tern_matrix& W, const uint16_t* x, int batch, uint
   a.unit = 1u;
   a.run = plan.run;
   a.kmax = plan.kmax;
+  a.early = (flags & TERN_GEMV_STATIC_WEIGHTS) ? 1 : 0;
   a.ws = plan.ws_bytes ? static_cast<float*>(workspace) : nullptr;
   a.counters = plan.ws_bytes ? reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + plan.ws_partial_bytes) : nullptr;
   if (plan.reg && W.layout == TERN_Q1_0_G128) {

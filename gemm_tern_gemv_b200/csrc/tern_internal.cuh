@@ -53,8 +53,9 @@ GemvPlan gemv_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms)
 // the GEMM kernel does not take.
 bool gemv_supported(int32_t layout, int64_t n, int64_t k, int64_t batch);
 
+// flags: TERN_GEMV_* bits of tern_gemv_ex (0 for tern_gemv).
 cudaError_t launch_gemv(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y,
-                        void* workspace, const GemvPlan& plan, cudaStream_t st);
+                        void* workspace, const GemvPlan& plan, cudaStream_t st, uint32_t flags = 0);
 
 // tern_gemv_noalloc's work after argument checks (scratch in a static device array).
 tern_status gemv_noalloc(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y, cudaStream_t st);

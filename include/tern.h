@@ -181,6 +181,20 @@ TERN_API size_t tern_gemv_workspace_bytes(const tern_matrix* W, int64_t batch);
 TERN_API tern_status tern_gemv(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y,
                       void* workspace, size_t workspace_bytes, void* stream);
 
+/* Flag of tern_gemv_ex: nothing that may still be running on the GPU when the call is made writes
+ * W's codes or scales (the usual case in a decode loop over fixed weights). The register-decode GEMV
+ * (batches 1-4 of Q2_0_g128, 1-2 of base-3, below 17 of Q1_0_g128) is then launched as a
+ * programmatic dependent of the preceding kernel on the stream: its CTAs may start as the preceding
+ * grid's CTAs leave their SMs and begin streaming W, while x, y and the workspace are still only
+ * touched after the preceding grid has completed. Other paths ignore the flag. */
+#define TERN_GEMV_STATIC_WEIGHTS 1u
+
+/* tern_gemv with flags (0 or TERN_GEMV_STATIC_WEIGHTS); same arguments, result and errors, plus
+ * TERN_ERR_INVALID_ARG for an unknown flag bit. This entry point is an engineering addition; the
+ * pages have no counterpart to it. */
+TERN_API tern_status tern_gemv_ex(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y,
+                                  void* workspace, size_t workspace_bytes, uint32_t flags, void* stream);
+
 /* Bytes of device memory tern_gemv_noalloc keeps for its split-K scratch (per GPU, for the
  * lifetime of the process). */
 #define TERN_GEMV_NOALLOC_SCRATCH_BYTES (8u << 20)

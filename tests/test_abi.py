@@ -92,6 +92,16 @@ def test_gemv_rejects_bad_matrix(lib, kw, status):
     assert st == status
 
 
+def test_gemv_ex_rejects_unknown_flags(lib):
+    m = _mat()
+    args = (ctypes.byref(m), ctypes.c_void_p(FAKE), 1, ctypes.c_void_p(FAKE), None, 0)
+    assert lib.tern_gemv_ex(*args, 2, None) == 1
+    assert lib.tern_gemv_ex(*args, 0x80000000, None) == 1
+    # a valid flag passes the flag check and stops at the next host-side check (missing workspace)
+    w = _mat(n=4096, k=4096, code_row_stride=1024, scale_row_stride=32)
+    assert lib.tern_gemv_ex(ctypes.byref(w), ctypes.c_void_p(FAKE), 1, ctypes.c_void_p(FAKE), None, 0, 1, None) == 4
+
+
 def test_gemv_rejects_bad_batch_and_buffers(lib):
     m = _mat()
     assert lib.tern_gemv(ctypes.byref(m), ctypes.c_void_p(FAKE), 0, ctypes.c_void_p(FAKE), None, 0, None) == 1
