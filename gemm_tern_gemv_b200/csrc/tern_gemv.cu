@@ -62,6 +62,7 @@ struct Args {
   int kmax;         // register kernel: partial-sum slots per tile and slice
   uint32_t unit;    // always 1 (see `mul` in the kernel)
   int early;        // register kernel: W may be read before earlier work on the stream completes
+  int local;        // register kernel: CTA-local reduction of whole tiles (no workspace)
 };
 
 // ---- small device helpers --------------------------------------------------------------------
@@ -597,15 +598,9 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(Args a) {
 // The MMA columns are (batch, group-within-window) pairs: a base-3 window touches three groups, so a
 // lane's four k-slots may belong to two groups and the activation fragments are stored per column.
 // A binary window holds four groups, so its eight columns carry two batch rows.
-#ifndef TERN_REG_WARPS
-#define TERN_REG_WARPS 16
-#endif
-#ifndef TERN_REG_CTAS_PER_SM
-#define TERN_REG_CTAS_PER_SM 1
-#endif
-constexpr int kSWarps = TERN_REG_WARPS;
-constexpr int kSThreads = kSWarps * 32;
-constexpr int kRegCtasPerSm = TERN_REG_CTAS_PER_SM;
+// Two CTA shapes, NW warps x CPS CTAs per SM: 16 x 1 puts all of an SM's warps on the few row tiles
+// of a small matrix; 8 x 2 (two independent CTAs per SM, each with its own fragment build and
+// reduction) is faster once there are several row tiles per CTA.
 constexpr int kWinBytes = 64;
 
 template <int LAYOUT> struct Lay;
@@ -641,9 +636,9 @@ __host__ __device__ constexpr uint32_t s_frag_window_bytes(int layout, int bs) {
 __host__ __device__ constexpr uint32_t s_stage_bytes(int layout, int rt) {
   return (uint32_t)rt * 16 * (kWinBytes + 16 * (layout == TERN_T3_5PB_G128 ? 2 : 1));
 }
-__host__ __device__ inline size_t s_smem_bytes(int layout, int rt, int stages, int gps, int bs) {
+__host__ __device__ inline size_t s_smem_bytes(int layout, int rt, int stages, int gps, int bs, int nw) {
   return (size_t)s_frag_window_bytes(layout, bs) * (s_windows(layout, gps) + 1) +
-         (size_t)kSWarps * stages * (s_stage_bytes(layout, rt) + 8) + 16;  // + full barriers, abort flag
+         (size_t)nw * stages * (s_stage_bytes(layout, rt) + 8) + 16;  // + full barriers, abort flag
 }
 
 __device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
@@ -719,24 +714,24 @@ __device__ __forceinline__ void s_frag_half(const Args& a, int g0, int kslice, i
   }
 }
 
-template <int LAYOUT, int BS>
+template <int LAYOUT, int BS, int NT>
 __device__ void s_build_frag(const Args& a, int g0, int ngroups, int nwin_alloc, uint8_t* frag) {
   constexpr uint32_t FW = s_frag_window_bytes(LAYOUT, BS);
   uint4* f4 = reinterpret_cast<uint4*>(frag);
   if (LAYOUT != TERN_T3_5PB_G128) {
     // every entry a data lane reads is written below (zero past the slice); only the zero block
-    for (int i = threadIdx.x; i < (int)(FW / 16); i += kSThreads)
+    for (int i = threadIdx.x; i < (int)(FW / 16); i += NT)
       f4[(size_t)nwin_alloc * FW / 16 + i] = make_uint4(0u, 0u, 0u, 0u);
   } else {
     // base-3 entries hold one group column each: the other columns must read as zero
-    for (int i = threadIdx.x; i < (int)((nwin_alloc + 1) * FW / 16); i += kSThreads) f4[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = threadIdx.x; i < (int)((nwin_alloc + 1) * FW / 16); i += NT) f4[i] = make_uint4(0u, 0u, 0u, 0u);
     __syncthreads();
   }
   uint16_t* fh = reinterpret_cast<uint16_t*>(frag);
   const int kslice = ngroups * kGroup;
   const int nwin = s_windows(LAYOUT, ngroups);
   const int items = nwin * 4 * a.batch * 2;
-  for (int e = threadIdx.x; e < items; e += kSThreads) {
+  for (int e = threadIdx.x; e < items; e += NT) {
     const int hf = e & 1, q = (e >> 1) & 3, rest = e >> 3;
     const int b = rest % a.batch, w = rest / a.batch;
     if (hf == 0) s_frag_half<LAYOUT, BS, 0>(a, g0, kslice, w, q, b, fh);
@@ -857,8 +852,8 @@ __device__ __forceinline__ void s_publish(const Args& a, const int (&tile)[2], c
 
 constexpr uint64_t kRegWaitLimitNs = 1000000000ull;  // 1 s: far beyond any healthy TMA latency
 
-template <int LAYOUT, int RT, int BS, int STAGES>
-__global__ void __launch_bounds__(kSThreads, kRegCtasPerSm)
+template <int LAYOUT, int RT, int BS, int STAGES, int NW, int CPS>
+__global__ void __launch_bounds__(NW * 32, CPS)
     gemv_reg_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales, Args a) {
   using L = Lay<LAYOUT>;
   constexpr int ROWS = RT * 16;
@@ -877,9 +872,9 @@ __global__ void __launch_bounds__(kSThreads, kRegCtasPerSm)
   uint8_t* frag = smem;
   uint8_t* rings = smem + (size_t)(nwin_alloc + 1) * FW;
   uint8_t* ring = rings + (size_t)warp * STAGES * STAGE;
-  uint64_t* full = reinterpret_cast<uint64_t*>(rings + (size_t)kSWarps * STAGES * STAGE) + warp * STAGES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(rings + (size_t)NW * STAGES * STAGE) + warp * STAGES;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(
-      reinterpret_cast<uint64_t*>(rings + (size_t)kSWarps * STAGES * STAGE) + kSWarps * STAGES);
+      reinterpret_cast<uint64_t*>(rings + (size_t)NW * STAGES * STAGE) + NW * STAGES);
 
   if (lane == 0) {
     for (int s = 0; s < STAGES; s++) sm100::mbar_init(full + s, 1);
@@ -893,12 +888,27 @@ __global__ void __launch_bounds__(kSThreads, kRegCtasPerSm)
   // (programmatic dependent launch; a no-op for plain launches).
   sm100::griddep_launch_dependents();
 
-  // this warp's run of (tile, window) units in the slice (empty past the last run); runs are dealt
-  // to CTAs round-robin so both CTAs on an SM, and all SMs, get the same number of runs (+-1)
-  const int wi = blockIdx.x + warp * gridDim.x;
-  const int units = a.tiles * nwin;
-  const int u_begin = min(wi * a.run, units);
-  const int u_end = min(u_begin + a.run, units);
+  // this warp's run of (tile, window) units in the slice (empty past the last run).
+  //   stream-K: runs of a.run units are dealt to CTAs round-robin, so both CTAs on an SM, and all SMs,
+  //     get the same number of runs (+-1); tiles shared by runs are summed through the workspace.
+  //   a.local: CTA c owns the whole tiles [t_lo, t_hi) (counts differ by at most one) and its warps
+  //     split their units into equal runs; shared tiles are summed in shared memory.
+  int wi, u_begin, u_end, t_lo = 0, t_hi = 0, lrun = 1, lbase = 0;
+  if (a.local) {
+    t_lo = (int)(((long long)blockIdx.x * a.tiles) / gridDim.x);
+    t_hi = (int)(((long long)(blockIdx.x + 1) * a.tiles) / gridDim.x);
+    const int ucta = (t_hi - t_lo) * nwin;
+    lrun = max(1, (ucta + NW - 1) / NW);
+    lbase = t_lo * nwin;
+    wi = warp;
+    u_begin = lbase + min(warp * lrun, ucta);
+    u_end = lbase + min(warp * lrun + lrun, ucta);
+  } else {
+    wi = blockIdx.x + warp * gridDim.x;
+    const int units = a.tiles * nwin;
+    u_begin = min(wi * a.run, units);
+    u_end = min(u_begin + a.run, units);
+  }
   const int total = u_end - u_begin;
   const int tile0 = u_begin / nwin, w0 = u_begin - tile0 * nwin;
 
@@ -932,7 +942,7 @@ __global__ void __launch_bounds__(kSThreads, kRegCtasPerSm)
   if (!a.early && lane == 0)
     for (int st = 0; st < STAGES && st < total; st++) issue_next();
 
-  s_build_frag<LAYOUT, BS>(a, g0, ngroups, nwin_alloc, frag);
+  s_build_frag<LAYOUT, BS, NW * 32>(a, g0, ngroups, nwin_alloc, frag);
 
   // B column of this lane and the fragment address it reads (zero block when it carries no data)
   int fb, fcol;
@@ -965,6 +975,8 @@ __global__ void __launch_bounds__(kSThreads, kRegCtasPerSm)
   const uint32_t lane_scale = kCodeBytes + g * (16 * L::SC);  // + (rt * 16 + 8 hr) * 16 * SC
   int c_tile = tile0, c_w = w0, c_slot = 0;
   int pend_tile[2] = {0, 0}, pend_contrib[2] = {0, 0}, npend = 0;  // partial tiles awaiting their count
+  float first_part[RT][2];  // a.local: partial of the run's first tile when that tile is shared
+  bool has_first = false;
   int st = 0;
   for (; st < total; st++) {
     if (!sm100::mbar_wait_bounded(full + c_slot, (st / STAGES) & 1, abort_flag, nullptr, 0u, kRegWaitLimitNs)) break;
@@ -1095,9 +1107,36 @@ __global__ void __launch_bounds__(kSThreads, kRegCtasPerSm)
     if (++c_slot == STAGES) c_slot = 0;
     if (++c_w == nwin || st == total - 1) {
       // end of this warp's run inside the tile: a tile covered by this run alone gets y now; a shared
-      // one gets this run's partial in the slot of its rank among the tile's runs
-      const int contributors = s_contributors<LAYOUT>(a, c_tile);
+      // one gets this run's partial in the slot of its rank among the tile's runs (workspace), or in
+      // this warp's first- or last-tile slot in shared memory (a.local)
+      int contributors;
+      if (a.local) {
+        const int rel0 = c_tile * nwin - lbase;
+        contributors = (rel0 + nwin - 1) / lrun - rel0 / lrun + 1;
+      } else {
+        contributors = s_contributors<LAYOUT>(a, c_tile);
+      }
       if (contributors == 1) {
+        s_store<LAYOUT, RT>(a, c_tile, -1, lane, acc);
+      } else if (a.local) {
+        // the partial of the run's first tile waits in registers; the last tile's is only reached at
+        // the run's last window, when every box of this warp's ring has been consumed, so it goes
+        // straight to the ring (partials: [first / last tile][lane][rt, hr] floats at the ring base)
+        if (c_tile == tile0) {
+#pragma unroll
+          for (int rt = 0; rt < RT; rt++) {
+            first_part[rt][0] = acc[rt][0];
+            first_part[rt][1] = acc[rt][1];
+          }
+          has_first = true;
+        } else {
+          float* dst = reinterpret_cast<float*>(ring) + (32 + lane) * (2 * RT);
+#pragma unroll
+          for (int rt = 0; rt < RT; rt++) {
+            dst[2 * rt] = acc[rt][0];
+            dst[2 * rt + 1] = acc[rt][1];
+          }
+        }
         s_store<LAYOUT, RT>(a, c_tile, -1, lane, acc);
       } else {
         const int seg = wi - (c_tile * nwin) / a.run;
@@ -1119,6 +1158,39 @@ __global__ void __launch_bounds__(kSThreads, kRegCtasPerSm)
     }
   }
   if (npend) s_publish<LAYOUT, RT>(a, pend_tile, pend_contrib, npend, lane);
+  if (a.local) {
+    if (has_first) {
+      float* dst = reinterpret_cast<float*>(ring) + lane * (2 * RT);
+#pragma unroll
+      for (int rt = 0; rt < RT; rt++) {
+        dst[2 * rt] = first_part[rt][0];
+        dst[2 * rt + 1] = first_part[rt][1];
+      }
+    }
+    // every run of the CTA has parked its shared-tile partials; each shared tile is summed by its first
+    // contributor, over the contributors in warp order (deterministic), and stored
+    __syncthreads();
+    for (int t = t_lo; t < t_hi; t++) {
+      const int rel0 = t * nwin - lbase;
+      if (rel0 / lrun != warp) continue;
+      const int wl = (rel0 + nwin - 1) / lrun;
+      if (wl == warp) continue;
+      float sum[RT][2];
+#pragma unroll
+      for (int rt = 0; rt < RT; rt++) sum[rt][0] = sum[rt][1] = 0.f;
+      for (int w = warp; w <= wl; w++) {
+        const int first = (lbase + w * lrun) / nwin;  // the first tile of warp w's run
+        const float* src = reinterpret_cast<const float*>(rings + (size_t)w * STAGES * STAGE) +
+                           ((t == first ? 0 : 32) + lane) * (2 * RT);
+#pragma unroll
+        for (int rt = 0; rt < RT; rt++) {
+          sum[rt][0] += src[2 * rt];
+          sum[rt][1] += src[2 * rt + 1];
+        }
+      }
+      s_store<LAYOUT, RT>(a, t, -1, lane, sum);
+    }
+  }
   // After a timeout, let the boxes still in flight land (again bounded in time) before the CTA's
   // shared memory is released.
   if (st < total) {
@@ -1175,20 +1247,20 @@ cudaError_t dispatch(const Args& a, int gx_hint, cudaStream_t st) {
   return cudaErrorInvalidValue;
 }
 
-template <int LAYOUT, int RT, int BS, int STAGES>
+template <int LAYOUT, int RT, int BS, int STAGES, int NW, int CPS>
 cudaError_t launch_reg(const CUtensorMap& tc, const CUtensorMap& ts, const Args& a, int grid_x, cudaStream_t st) {
-  const size_t smem = s_smem_bytes(LAYOUT, RT, STAGES, a.gps, BS);
-  auto kern = gemv_reg_kernel<LAYOUT, RT, BS, STAGES>;
+  const size_t smem = s_smem_bytes(LAYOUT, RT, STAGES, a.gps, BS, NW);
+  auto kern = gemv_reg_kernel<LAYOUT, RT, BS, STAGES, NW, CPS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if (!a.early) {
-    kern<<<dim3(grid_x, a.splits), kSThreads, smem, st>>>(tc, ts, a);
+    kern<<<dim3(grid_x, a.splits), NW * 32, smem, st>>>(tc, ts, a);
     return cudaGetLastError();
   }
   // programmatic dependent launch: the grid may start while the preceding kernel finishes
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid_x, a.splits);
-  cfg.blockDim = dim3(kSThreads);
+  cfg.blockDim = dim3(NW * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -1222,7 +1294,14 @@ bool use_reg_kernel(int32_t layout, int64_t n, int64_t k, int64_t batch) {
   return layout == TERN_Q2_0_G128 ? batch <= 4 : layout == TERN_Q1_0_G128 ? true : batch <= 2;
 }
 
-cudaError_t dispatch_reg(const tern_matrix& W, const Args& a, int grid_x, cudaStream_t st) {
+template <int LAYOUT, int BS, int STAGES>
+cudaError_t launch_shape(const CUtensorMap& tc, const CUtensorMap& ts, const Args& a, int grid_x, int warps,
+                         cudaStream_t st) {
+  if (warps == 8) return launch_reg<LAYOUT, kRegRT, BS, STAGES, 8, 2>(tc, ts, a, grid_x, st);
+  return launch_reg<LAYOUT, kRegRT, BS, STAGES, 16, 1>(tc, ts, a, grid_x, st);
+}
+
+cudaError_t dispatch_reg(const tern_matrix& W, const Args& a, int grid_x, int warps, cudaStream_t st) {
   // tensor maps: codes [n][row data bytes] in boxes of 64 B x tile rows; scales [n][groups] in boxes
   // of 8 (Q2, binary) or 16 (base-3) groups x tile rows
   const bool q2 = W.layout == TERN_Q2_0_G128, q1 = W.layout == TERN_Q1_0_G128;
@@ -1235,28 +1314,29 @@ cudaError_t dispatch_reg(const tern_matrix& W, const Args& a, int grid_x, cudaSt
                (uint64_t)W.scale_row_stride * 2, q2 || q1 ? 8 : 16, 16 * kRegRT, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   if (q1) {
-    if (a.batch == 1) return launch_reg<TERN_Q1_0_G128, kRegRT, 1, kRegStagesQ2>(tc, ts, a, grid_x, st);
-    return launch_reg<TERN_Q1_0_G128, kRegRT, 2, kRegStagesQ2>(tc, ts, a, grid_x, st);
+    if (a.batch == 1) return launch_shape<TERN_Q1_0_G128, 1, kRegStagesQ2>(tc, ts, a, grid_x, warps, st);
+    return launch_shape<TERN_Q1_0_G128, 2, kRegStagesQ2>(tc, ts, a, grid_x, warps, st);
   }
   if (q2) {
     switch (bs_for(a.batch)) {
-      case 1: return launch_reg<TERN_Q2_0_G128, kRegRT, 1, kRegStagesQ2>(tc, ts, a, grid_x, st);
-      case 2: return launch_reg<TERN_Q2_0_G128, kRegRT, 2, kRegStagesQ2>(tc, ts, a, grid_x, st);
-      default: return launch_reg<TERN_Q2_0_G128, kRegRT, 4, kRegStagesQ2>(tc, ts, a, grid_x, st);
+      case 1: return launch_shape<TERN_Q2_0_G128, 1, kRegStagesQ2>(tc, ts, a, grid_x, warps, st);
+      case 2: return launch_shape<TERN_Q2_0_G128, 2, kRegStagesQ2>(tc, ts, a, grid_x, warps, st);
+      default: return launch_shape<TERN_Q2_0_G128, 4, kRegStagesQ2>(tc, ts, a, grid_x, warps, st);
     }
   }
-  if (a.batch == 1) return launch_reg<TERN_T3_5PB_G128, kRegRT, 1, kRegStagesT3>(tc, ts, a, grid_x, st);
-  return launch_reg<TERN_T3_5PB_G128, kRegRT, 2, kRegStagesT3>(tc, ts, a, grid_x, st);
+  if (a.batch == 1) return launch_shape<TERN_T3_5PB_G128, 1, kRegStagesT3>(tc, ts, a, grid_x, warps, st);
+  return launch_shape<TERN_T3_5PB_G128, 2, kRegStagesT3>(tc, ts, a, grid_x, warps, st);
 }
 
 }  // namespace
 
-// Register kernel: the fewest K slices whose activation fragments leave room for the target number
-// of CTAs per SM, one full wave of CTAs, and the slice's (tile, window) units spread evenly over
-// the warps.
-static GemvPlan reg_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
+// Register kernel with NW warps x CPS CTAs per SM: the fewest K slices whose activation fragments
+// leave room for CPS CTAs per SM, one full wave of CTAs, and the slice's (tile, window) units spread
+// evenly over the warps.
+static GemvPlan reg_plan_shape(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms, int nw, int cps) {
   GemvPlan p{};
   p.reg = true;
+  p.warps = nw;
   if (layout == TERN_Q1_0_G128) batch = std::min<int64_t>(batch, kBinChunk);  // one launch per pair of rows
   const int groups = (int)(k / kGroup);
   // K-slice granularity in groups: one window
@@ -1264,14 +1344,14 @@ static GemvPlan reg_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, in
   const int units = (groups + unit - 1) / unit;
   const int stages = layout == TERN_T3_5PB_G128 ? kRegStagesT3 : kRegStagesQ2;
   const int bs = bs_for(batch);
-  // shared memory of one CTA when kRegCtasPerSm of them share an SM (228 KB, 1 KB reserved each)
-  const size_t cap = (size_t)(228 / kRegCtasPerSm - 1) * 1024;
+  // shared memory of one CTA when cps of them share an SM (228 KB, 1 KB reserved each)
+  const size_t cap = (size_t)(228 / cps - 1) * 1024;
   int upc = units;
-  while (upc > 1 && s_smem_bytes(layout, kRegRT, stages, upc * unit, bs) > cap) upc = (upc + 1) / 2;
+  while (upc > 1 && s_smem_bytes(layout, kRegRT, stages, upc * unit, bs, nw) > cap) upc = (upc + 1) / 2;
   const int splits = (units + upc - 1) / upc;
   const int gps = std::min(groups, upc * unit);
-  const size_t smem = s_smem_bytes(layout, kRegRT, stages, gps, bs);
-  const int per_sm = std::max(1, std::min(kRegCtasPerSm, (int)(227 * 1024 / (smem + 1024))));
+  const size_t smem = s_smem_bytes(layout, kRegRT, stages, gps, bs, nw);
+  const int per_sm = std::max(1, std::min(cps, (int)(227 * 1024 / (smem + 1024))));
   p.rows_per_cta = 16 * kRegRT;
   p.row_blocks = (int)((n + p.rows_per_cta - 1) / p.rows_per_cta);
   p.splits = splits;
@@ -1279,18 +1359,42 @@ static GemvPlan reg_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, in
   const int nwin_full = s_windows(layout, gps);
   const int64_t u_full = (int64_t)p.row_blocks * nwin_full;
   // runs of `run` units, at most one per warp of a full wave; the longest run sets the time
-  const int64_t warps = (int64_t)std::max(1, (sms * per_sm) / splits) * kSWarps;
+  const int64_t warps = (int64_t)std::max(1, (sms * per_sm) / splits) * nw;
   p.run = (int)std::max<int64_t>(1, (u_full + warps - 1) / warps);
   const int64_t runs = (u_full + p.run - 1) / p.run;
   // a full wave of CTAs whenever there are runs for it (runs are dealt round-robin over CTAs)
   p.grid_x = (int)std::min<int64_t>(std::max(1, (sms * per_sm) / splits), runs);
   p.kmax = (nwin_full - 1 + p.run - 1) / p.run + 1;  // runs that can touch one tile
+  // CTA-local reduction when K is one slice and it costs each warp at most one window more than
+  // stream-K: no workspace, and the global partial-sum round trips (store, fence, counter, reload)
+  // leave the end of the kernel.
+  if (splits == 1) {
+    const int64_t grid_l = std::min<int64_t>(p.row_blocks, (int64_t)sms * per_sm);
+    const int64_t tmax = (p.row_blocks + grid_l - 1) / grid_l;
+    const int64_t lwin = (tmax * nwin_full + nw - 1) / nw;
+    if (lwin <= p.run + 1) {
+      p.local = true;
+      p.grid_x = (int)grid_l;
+      return p;
+    }
+  }
   const bool whole_tiles = splits == 1 && p.run % nwin_full == 0;
   if (!whole_tiles) {
     p.ws_partial_bytes = (size_t)splits * p.kmax * batch * n * sizeof(float);
     p.ws_bytes = (p.ws_partial_bytes + (size_t)p.row_blocks * sizeof(int) + 15) / 16 * 16;
   }
   return p;
+}
+
+// The CTA shape for a register-kernel launch: 8 warps x 2 CTAs per SM once there are at least four row
+// tiles per SM and K still fits one slice in the smaller CTA; 16 warps x 1 CTA otherwise.
+static GemvPlan reg_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
+  const int64_t tiles = (n + 16 * kRegRT - 1) / (16 * kRegRT);
+  if (tiles >= 4 * (int64_t)sms) {
+    const GemvPlan p = reg_plan_shape(layout, n, k, batch, sms, 8, 2);
+    if (p.splits == 1) return p;
+  }
+  return reg_plan_shape(layout, n, k, batch, sms, 16, 1);
 }
 
 // Batches from this size on run on the tcgen05 prefill GEMM kernel: its tensor core takes the decoded
@@ -1357,6 +1461,7 @@ cudaError_t launch_gemv(const tern_matrix& W, const uint16_t* x, int batch, uint
   a.run = plan.run;
   a.kmax = plan.kmax;
   a.early = (flags & TERN_GEMV_STATIC_WEIGHTS) ? 1 : 0;
+  a.local = plan.local ? 1 : 0;
   a.ws = plan.ws_bytes ? static_cast<float*>(workspace) : nullptr;
   a.counters = plan.ws_bytes ? reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + plan.ws_partial_bytes) : nullptr;
   if (plan.reg && W.layout == TERN_Q1_0_G128) {
@@ -1366,12 +1471,12 @@ cudaError_t launch_gemv(const tern_matrix& W, const uint16_t* x, int batch, uint
       a.batch = std::min(kBinChunk, batch - b0);
       a.x = x + (int64_t)b0 * W.k;
       a.y = y + (int64_t)b0 * W.n;
-      const cudaError_t e = dispatch_reg(W, a, plan.grid_x, st);
+      const cudaError_t e = dispatch_reg(W, a, plan.grid_x, plan.warps, st);
       if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
   }
-  if (plan.reg) return dispatch_reg(W, a, plan.grid_x, st);
+  if (plan.reg) return dispatch_reg(W, a, plan.grid_x, plan.warps, st);
   const int gx_hint = (plan.row_blocks + kWarps - 1) / kWarps;
   if (W.layout == TERN_Q2_0_G128) return dispatch<TERN_Q2_0_G128>(a, gx_hint, st);
   return dispatch<TERN_T3_5PB_G128>(a, gx_hint, st);

@@ -45,6 +45,8 @@ struct GemvPlan {
   int grid_x;           // register kernel: CTAs per K slice
   int run;              // register kernel: (tile, window) units per warp run
   int kmax;             // register kernel: partial-sum slots per tile and K slice
+  bool local;           // register kernel: each CTA owns whole row tiles, summed in shared memory
+  int warps;            // register kernel: warps per CTA (16, one CTA per SM; or 8, two per SM)
   size_t ws_partial_bytes;  // fp32 partial sums [splits * slots][batch][n]
   size_t ws_bytes;          // partials + one int32 counter per row block, rounded to 16
 };

@@ -98,7 +98,7 @@ def test_gemv_ex_rejects_unknown_flags(lib):
     assert lib.tern_gemv_ex(*args, 2, None) == 1
     assert lib.tern_gemv_ex(*args, 0x80000000, None) == 1
     # a valid flag passes the flag check and stops at the next host-side check (missing workspace)
-    w = _mat(n=4096, k=4096, code_row_stride=1024, scale_row_stride=32)
+    w = _mat(n=5120, k=17408, code_row_stride=4352, scale_row_stride=136)
     assert lib.tern_gemv_ex(ctypes.byref(w), ctypes.c_void_p(FAKE), 1, ctypes.c_void_p(FAKE), None, 0, 1, None) == 4
 
 
@@ -112,8 +112,8 @@ def test_gemv_rejects_bad_batch_and_buffers(lib):
 
 
 def test_gemv_workspace_size_and_rejection(lib):
-    # a narrow matrix needs split-K workspace; too little is refused before any launch
-    m = _mat(n=4096, k=4096, code_row_stride=1024, scale_row_stride=32)
+    # a narrow matrix with a long K needs split-K workspace; too little is refused before any launch
+    m = _mat(n=5120, k=17408, code_row_stride=4352, scale_row_stride=136)
     need = lib.tern_gemv_workspace_bytes(ctypes.byref(m), 1)
     assert need > 0 and need % 16 == 0
     assert lib.tern_gemv(ctypes.byref(m), ctypes.c_void_p(FAKE), 1, ctypes.c_void_p(FAKE), None, 0, None) == 4
@@ -121,9 +121,14 @@ def test_gemv_workspace_size_and_rejection(lib):
                          ctypes.c_void_p(FAKE), need - 16, None) == 4
     assert lib.tern_gemv(ctypes.byref(m), ctypes.c_void_p(FAKE), 1, ctypes.c_void_p(FAKE),
                          ctypes.c_void_p(FAKE + 8), need, None) == 3
-    # a matrix of one 128-weight group per row is never split and needs none
+    # a matrix of one 128-weight group per row is never split and needs none; neither do the 8B-class
+    # decode shapes at batch 1, whose tiles are summed inside each CTA
     one = _mat(n=4096, k=128, code_row_stride=32, scale_row_stride=8)
     assert lib.tern_gemv_workspace_bytes(ctypes.byref(one), 1) == 0
+    for layout, rb in ((1, 1024), (2, 832), (3, 512)):
+        for n in (4096, 24576):
+            sq = _mat(layout=layout, n=n, k=4096, code_row_stride=rb, scale_row_stride=32)
+            assert lib.tern_gemv_workspace_bytes(ctypes.byref(sq), 1) == 0
     # the size is a pure function of the arguments; batch outside 1..64 gives 0
     big = _mat(n=151936, k=4096, code_row_stride=1024, scale_row_stride=32)
     assert lib.tern_gemv_workspace_bytes(ctypes.byref(big), 1) == lib.tern_gemv_workspace_bytes(ctypes.byref(big), 1)
@@ -135,7 +140,7 @@ def test_gemv_workspace_size_and_rejection(lib):
 def test_binary_gemv_workspace_is_that_of_two_rows(lib):
     # the binary register kernel runs batch rows in pairs, one launch after another on the stream,
     # so every batch below the GEMM's reuses the workspace of a two-row launch
-    m = _mat(layout=3, n=4096, k=4096, code_row_stride=512, scale_row_stride=32)
+    m = _mat(layout=3, n=5120, k=17408, code_row_stride=2176, scale_row_stride=136)
     two = lib.tern_gemv_workspace_bytes(ctypes.byref(m), 2)
     assert two > 0
     for b in (3, 7, 16):

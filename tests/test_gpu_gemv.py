@@ -80,7 +80,7 @@ def test_activation_dynamic_range():
 
 @pytest.mark.parametrize("layout", LAYOUTS)
 def test_split_k_deterministic_and_workspace_reuse(layout):
-    n, k, batch = 4096, 4096, 2
+    n, k, batch = 1000, 17408, 2
     codes, s, x = workload(layout, n, k, batch, seed=11)
     W = T.from_packed(torch.from_numpy(codes).cuda(), torch.from_numpy(s).cuda(), layout, k)
     ws = T.gemv_workspace(W, batch)
@@ -94,6 +94,24 @@ def test_split_k_deterministic_and_workspace_reuse(layout):
     rows = sample_rows(n, 256, 1)
     y_ref, a = O.gemv(codes, s, x, layout, k, rows=rows)
     check_product(y1.cpu().numpy()[:, rows], y_ref, a, "split-K")
+
+
+@pytest.mark.parametrize("layout", LAYOUTS)
+@pytest.mark.parametrize("n,k,batch", [(4096, 4096, 1), (24576, 4096, 2), (4096, 12288, 1), (300, 2048, 1)])
+def test_cta_local_reduction_is_deterministic(layout, n, k, batch):
+    # these shapes sum each row tile inside one CTA (no workspace); repeated calls agree bit for bit
+    codes, s, x = workload(layout, n, k, batch, seed=n + k + 3)
+    W = T.from_packed(torch.from_numpy(codes).cuda(), torch.from_numpy(s).cuda(), layout, k)
+    xg = torch.from_numpy(x).cuda()
+    if layout != T.T3_5PB_G128 or k == 4096:
+        assert T.gemv_workspace(W, batch) is None
+    y1 = T.gemv(W, xg).clone()
+    y2 = T.gemv(W, xg, static_weights=True).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    rows = sample_rows(n, 384, 5)
+    y_ref, a = O.gemv(codes, s, x, layout, k, rows=rows)
+    check_product(y1.cpu().numpy()[:, rows], y_ref, a, "CTA-local reduction")
 
 
 # ---------------------------------------------------------------- the workload configurations

@@ -53,7 +53,7 @@ def test_chain_of_dependent_calls_matches_plain_calls(layout, batch):
 
 @pytest.mark.parametrize("layout", LAYOUTS)
 def test_back_to_back_calls_share_one_workspace(layout):
-    n, k, batch = 4096, 4096, 1
+    n, k, batch = 1000, 17408, 1
     W, codes, s = _mat(layout, n, k, 50)
     ws = T.gemv_workspace(W, batch)
     assert ws is not None
