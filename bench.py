@@ -442,7 +442,7 @@ def measure_extras(torch, T, dev, peaks, stream):
 
     # LM head (base-3) and 27B batched GEMVs; weights larger than L2, re-read each launch
     cases = [("lm_head_t3", T.T3_5PB_G128, 151936, 4096, b) for b in (1, 8)]
-    # the binary layout on the 8B shapes: batch 1-2 is one launch, larger batches one launch per pair
+    # the binary layout on the 8B shapes: batch 1-2 is one register-kernel launch, 3-4 two, 5 and up the GEMM
     for (n, k) in LAYER_SET:
         for b in (1, 2, 4, 16):
             cases.append((f"8b_q1_{n}x{k}", T.Q1_0_G128, n, k, b))

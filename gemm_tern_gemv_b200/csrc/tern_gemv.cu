@@ -1401,14 +1401,20 @@ static GemvPlan reg_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, in
 // weights at a fixed rate whatever the number of tokens sharing them, which beats the mma.sync
 // kernels once a weight serves this many rows of x.
 constexpr int kGemmMinBatch = 17;
+// The binary register kernel takes two rows of x per launch, so from this batch on the GEMM kernel
+// (one pass over W) is the faster of the two.
+constexpr int kGemmMinBatchBinary = 5;
+static bool use_gemm(int32_t layout, int64_t n, int64_t batch) {
+  return n % 8 == 0 && batch >= (layout == TERN_Q1_0_G128 ? kGemmMinBatchBinary : kGemmMinBatch);
+}
 
 bool gemv_supported(int32_t layout, int64_t n, int64_t k, int64_t batch) {
   if (layout != TERN_Q1_0_G128) return true;
-  return (batch >= kGemmMinBatch && n % 8 == 0) || use_reg_kernel(layout, n, k, batch);
+  return use_gemm(layout, n, batch) || use_reg_kernel(layout, n, k, batch);
 }
 
 GemvPlan gemv_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
-  if (batch >= kGemmMinBatch && n % 8 == 0) {
+  if (use_gemm(layout, n, batch)) {
     GemvPlan p{};
     p.gemm = true;
     p.splits = 1;

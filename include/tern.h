@@ -167,7 +167,8 @@ TERN_API size_t tern_gemv_workspace_bytes(const tern_matrix* W, int64_t batch);
 /* y[b][n] = sum_g s[n][g] * sum_{k in group g} t[n][k] * x[b][k] for b < batch; fp32
  * accumulation, fp16 result. Small batches run on mma.sync kernels that decode the codes in
  * registers; batches of 17 or more with n % 8 == 0 run on the tcgen05 kernel of tern_gemm (no
- * workspace). A Q1_0_g128 batch below that runs as one register-kernel launch per two rows of x.
+ * workspace); so do Q1_0_g128 batches of 5 or more with n % 8 == 0. Other Q1_0_g128 batches run
+ * as one register-kernel launch per two rows of x.
  * The result of a call depends only on (W, x, batch) and the device.
  *   x          device fp16 [batch][k], contiguous
  *   y          device fp16 [batch][n], contiguous
@@ -183,7 +184,7 @@ TERN_API tern_status tern_gemv(const tern_matrix* W, const uint16_t* x, int64_t 
 
 /* Flag of tern_gemv_ex: nothing that may still be running on the GPU when the call is made writes
  * W's codes or scales (the usual case in a decode loop over fixed weights). The register-decode GEMV
- * (batches 1-4 of Q2_0_g128, 1-2 of base-3, below 17 of Q1_0_g128) is then launched as a
+ * (batches 1-4 of Q2_0_g128, 1-2 of base-3, those of Q1_0_g128 not taken by the GEMM) is then launched as a
  * programmatic dependent of the preceding kernel on the stream: its CTAs may start as the preceding
  * grid's CTAs leave their SMs and begin streaming W, while x, y and the workspace are still only
  * touched after the preceding grid has completed. Other paths ignore the flag. */

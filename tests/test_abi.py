@@ -143,9 +143,12 @@ def test_binary_gemv_workspace_is_that_of_two_rows(lib):
     m = _mat(layout=3, n=5120, k=17408, code_row_stride=2176, scale_row_stride=136)
     two = lib.tern_gemv_workspace_bytes(ctypes.byref(m), 2)
     assert two > 0
-    for b in (3, 7, 16):
+    for b in (3, 4):
         assert lib.tern_gemv_workspace_bytes(ctypes.byref(m), b) == two
-    assert lib.tern_gemv_workspace_bytes(ctypes.byref(m), 17) == 0  # the GEMM kernel takes it
+    for b in (5, 16, 17):  # the GEMM kernel takes binary batches from 5 on (n % 8 == 0)
+        assert lib.tern_gemv_workspace_bytes(ctypes.byref(m), b) == 0
+    odd = _mat(layout=3, n=5121, k=17408, code_row_stride=2176, scale_row_stride=136)
+    assert lib.tern_gemv_workspace_bytes(ctypes.byref(odd), 16) == lib.tern_gemv_workspace_bytes(ctypes.byref(odd), 2)
 
 
 def test_pack_unpack_gemm_reject(lib):
