@@ -479,20 +479,31 @@ def measure_extras(torch, T, dev, peaks, stream):
     cache.clear()
     torch.cuda.empty_cache()
 
-    # transposed product dx = W^T dy (STE backward) on the 8B shapes, batch 1
+    # transposed product dx = W^T dy (STE backward) on the 8B shapes, batch 1; weight copies past L2
     for layout, lname in ((T.Q2_0_G128, "q2"), (T.T3_5PB_G128, "t3"), (T.Q1_0_G128, "q1")):
         for (n, k) in ((24576, 4096), (4096, 12288)):
-            Wt = make_weights(torch, T, n, k, layout, 6, dev)
+            wbytes = n * T.row_bytes(layout, k) + n * (k // GROUP) * 2
+            copies = max(2, min(64, -(-300_000_000 // wbytes)))
+            Wts = [make_weights(torch, T, n, k, layout, 6 + c, dev) for c in range(copies)]
             dy = torch.randn((1, n), device=dev).to(torch.float16)
             dxo = torch.empty((1, k), dtype=torch.float16, device=dev)
-            nbw = int(T.lib().tern_gemv_t_workspace_bytes(ctypes.byref(Wt.c()), 1))
+            nbw = int(T.lib().tern_gemv_t_workspace_bytes(ctypes.byref(Wts[0].c()), 1))
             wsv = torch.empty(max(nbw, 16), dtype=torch.uint8, device=dev)
-            ms = timed(lambda: T.gemv_t(Wt, dy, dx=dxo, workspace=wsv if nbw else None), 20)
+            it = [0]
+
+            def ft():
+                c = it[0] % len(Wts)
+                it[0] += 1
+                T.gemv_t(Wts[c], dy, dx=dxo, workspace=wsv if nbw else None)
+            ms = timed(ft, 20)
             nb = algorithmic_bytes(layout, n, k, 1)
             res[f"gemv_t_{lname}_{n}x{k}_b1"] = {"GB/s": round(nb / (ms * 1e-3) / 1e9, 1),
                                                  "frac_hbm": round(nb / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-                                                 "us": round(ms * 1e3, 2), "note": "L2-warm (one weight copy)"}
-            del Wt
+                                                 "us": round(ms * 1e3, 2),
+                                                 "note": f"{copies} weight copies (HBM-cold); partials "
+                                                         f"{nbw / 1e6:.1f} MB written and re-read"}
+            del Wts
+            torch.cuda.empty_cache()
 
     # activation-side block Hadamard rotation (sign flip + FWHT per 1024-block) in front of a GEMV
     signs = torch.where(torch.rand(1024, device=dev) < 0.5, -1, 1).to(torch.int8)

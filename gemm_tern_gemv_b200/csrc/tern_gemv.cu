@@ -35,6 +35,7 @@
 
 #include "sm100.cuh"
 #include "tern_internal.cuh"
+#include "tern_t3.cuh"
 
 namespace tern {
 namespace {
@@ -653,23 +654,6 @@ __device__ __forceinline__ uint32_t lds16(uint32_t addr) {
   return v;
 }
 
-// Base-3 word (bytes b0..b3) -> 10 A registers: o[5h + i] = (2 t of digit 4 - i of byte h,
-// same digit of byte 2 + h) as an fp16 pair.
-__device__ __forceinline__ void dec_t3_word(uint32_t w, uint32_t k0, uint32_t (&o)[10]) {
-#pragma unroll
-  for (int h = 0; h < 2; h++) {
-    const uint32_t V = h ? __byte_perm(w, 0u, 0x4341) : (w & 0x00FF00FFu);
-    uint32_t R = V * 202u + k0;
-    o[5 * h] = R & 0xC000C000u;
-    R = (R & 0x3FC03FC0u) * 3u + 0xC000C000u;
-    o[5 * h + 1] = R & 0xC000C000u;
-#pragma unroll
-    for (int i = 2; i < 5; i++) {
-      R = (R - o[5 * h + i - 1]) * 3u + 0xC000C000u;
-      o[5 * h + i] = R & 0xC000C000u;
-    }
-  }
-}
 
 // Activation fragments of one K slice, one entry (uint2 = the lane's b0, b1) per
 // [window][mma j / 2][batch slot][column c < C][q][j % 2], so a lane reads two MMAs' worth with one

@@ -3,98 +3,149 @@
 // 파인튜닝", molayo1419.me, paragraph "그것을 파인튜닝하는 방법": gradients flow through the
 // ternarized forward to the latent weights and the layer input).
 //
-// The contraction runs over the rows of W, so a warp reads whole rows: CTA (column block, row slice)
-// covers 64 code bytes of every row of its slice (256 columns of Q2_0_g128, 320 of base-3, 512 of
-// the binary Q1_0_g128); thread t owns byte t % 64 of rows t / 64, t / 64 + 4, ... and accumulates its
-// 4, 5 or 8 columns for every batch row in fp32 with s * dy formed once per row. The four row phases
-// of a CTA are summed through shared memory in two halving steps; row slices write fp32 partials that a second kernel sums in slice order
-// (deterministic), or the single slice stores dx directly.
+// The contraction runs over the rows of W, so the kernel streams whole rows with vector loads:
+//   * A warp covers a column block of 32 x LB bytes of every row it reads (LB = 16 / B bytes per lane,
+//     8 / B for the binary layout, B = the batch rounded up to 1, 2, 4 or 8), one LB-byte load per lane
+//     and row. Each lane keeps fp32 accumulators for its 64 (Q2_0_g128, binary) or 80 (base-3) / B
+//     columns and all B batch rows.
+//   * Decode straight to fp32: a two's-complement field moved to bits 30..31 of a float is +-2.0 or 0
+//     (sign and exponent MSB), so a multiply (the shift) and a mask give 2t exactly; a binary sign bit
+//     moved to bit 31 and XOR-ed with 0xC0000000 gives +-2.0. The FFMA multiplies by s * dy / 2, which
+//     is exact in fp32, so every product is exact and only the fp32 sums round.
+//   * The 8 warps of a CTA read interleaved rows of the same column block and are summed through
+//     shared memory in warp order; row slices write fp32 partials that a second kernel sums in slice
+//     order (deterministic), or the single slice stores dx directly.
 #include <cuda_fp16.h>
 
 #include "tern_internal.cuh"
+#include "tern_t3.cuh"
 
 namespace tern {
 namespace {
 
-constexpr int kTThreads = 256;
-constexpr int kTBytes = 64;  // code bytes of a row per column block
+constexpr int kTWarps = 8;
+constexpr int kTThreads = kTWarps * 32;
 
 template <int LAYOUT> constexpr int cols_per_byte() {
   return LAYOUT == TERN_Q2_0_G128 ? 4 : LAYOUT == TERN_Q1_0_G128 ? 8 : 5;
 }
-constexpr int kPhases = kTThreads / kTBytes;
+template <int LAYOUT, int B> constexpr int lane_bytes() { return (LAYOUT == TERN_Q1_0_G128 ? 8 : 16) / B; }
+template <int LAYOUT, int B> constexpr size_t red_bytes() {
+  return (size_t)kTWarps * 32 * lane_bytes<LAYOUT, B>() * cols_per_byte<LAYOUT>() * B * sizeof(float);
+}
 
-template <int LAYOUT, int BATCH>
+// The LB code bytes of a lane as little-endian 32-bit words (bytes past LB read as zero).
+template <int LB>
+__device__ __forceinline__ void load_codes(const uint8_t* p, uint32_t (&w)[(LB + 3) / 4]) {
+  if constexpr (LB == 16) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  } else if constexpr (LB == 8) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+    w[0] = v.x; w[1] = v.y;
+  } else if constexpr (LB == 4) {
+    w[0] = __ldg(reinterpret_cast<const uint32_t*>(p));
+  } else if constexpr (LB == 2) {
+    w[0] = __ldg(reinterpret_cast<const unsigned short*>(p));
+  } else {
+    w[0] = __ldg(p);
+  }
+}
+
+template <int LAYOUT, int B>
 __global__ void __launch_bounds__(kTThreads) gemv_t_kernel(const uint8_t* __restrict__ codes, int64_t cstride,
                                                            const uint16_t* __restrict__ scales, int64_t sstride,
                                                            const uint16_t* __restrict__ dy, int batch, int64_t n,
-                                                           int64_t k, int64_t rows_per_slice, float* part,
-                                                           uint16_t* dx) {
-  constexpr int C = cols_per_byte<LAYOUT>();
-  __shared__ float red[kPhases / 2][kTBytes * C][BATCH];
-  const int t = threadIdx.x, phase = t / kTBytes, byte = t % kTBytes;
-  const int64_t col0 = (int64_t)blockIdx.x * kTBytes * C + (int64_t)byte * C;  // first column of this byte
+                                                           int64_t k, int64_t row_bytes, int64_t rows_per_slice,
+                                                           float* part, uint16_t* dx) {
+  constexpr int LB = lane_bytes<LAYOUT, B>();
+  constexpr int CPB = cols_per_byte<LAYOUT>();
+  constexpr int CL = LB * CPB;  // columns of one lane
+  constexpr int NWD = (LB + 3) / 4;
+  extern __shared__ float red[];  // [warp][lane * CL + column][B]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t byte0 = ((int64_t)blockIdx.x * 32 + lane) * LB;  // this lane's first byte of a row
+  const int64_t col0 = byte0 * CPB;
   const int64_t n0 = (int64_t)blockIdx.y * rows_per_slice;
   const int64_t n1 = n0 + rows_per_slice < n ? n0 + rows_per_slice : n;
-  const int64_t byte_off = (int64_t)blockIdx.x * kTBytes + byte;
-  const int64_t data_bytes = LAYOUT == TERN_Q2_0_G128 ? k / 4 : LAYOUT == TERN_Q1_0_G128 ? k / 8 : (k + 4) / 5;
-  // groups of this byte's columns (a base-3 byte can straddle two 128-column groups)
-  const int64_t g_first = col0 / kGroup, g_last = (col0 + C - 1) / kGroup;
-  float acc[C][BATCH];
+  const int64_t groups = k / kGroup;
+  // a base-3 lane's 80 columns can straddle two groups: columns before `split` use the first scale
+  const int64_t g_first = col0 / kGroup;
+  const int64_t g_last = (col0 + CL - 1) / kGroup < groups ? (col0 + CL - 1) / kGroup : g_first;
+  const int split = (int)((g_first + 1) * kGroup - col0);
+
+  float acc[CL][B];
 #pragma unroll
-  for (int i = 0; i < C; i++)
+  for (int c = 0; c < CL; c++)
 #pragma unroll
-    for (int b = 0; b < BATCH; b++) acc[i][b] = 0.f;
-  if (byte_off < data_bytes) {
-    for (int64_t r = n0 + phase; r < n1; r += kTThreads / kTBytes) {
-      uint32_t v = __ldg(codes + r * cstride + byte_off);
+    for (int b = 0; b < B; b++) acc[c][b] = 0.f;
+
+  // byte0 and row_bytes are multiples of LB, so a lane with byte0 < row_bytes reads inside the row
+  if (byte0 < row_bytes && g_first < groups) {
+    const uint32_t k0 = (130u | (130u << 16)) + 0xC000C000u;
+    for (int64_t r = n0 + warp; r < n1; r += kTWarps) {
+      uint32_t w[NWD];
+      load_codes<LB>(codes + r * cstride + byte0, w);
       const float s0 = __half2float(__ushort_as_half(__ldg(scales + r * sstride + g_first)));
-      const float s1 = (g_last != g_first && g_last < k / kGroup)
-                           ? __half2float(__ushort_as_half(__ldg(scales + r * sstride + g_last))) : s0;
-      float d[BATCH];
+      const float s1 = g_last != g_first ? __half2float(__ushort_as_half(__ldg(scales + r * sstride + g_last))) : s0;
+      float sd0[B], sd1[B];
 #pragma unroll
-      for (int b = 0; b < BATCH; b++) d[b] = b < batch ? __half2float(__ushort_as_half(__ldg(dy + (int64_t)b * n + r))) : 0.f;
+      for (int b = 0; b < B; b++) {
+        const float d = b < batch ? __half2float(__ushort_as_half(__ldg(dy + (int64_t)b * n + r))) : 0.f;
+        sd0[b] = 0.5f * s0 * d;  // exact: products of fp16 values fit fp32
+        sd1[b] = 0.5f * s1 * d;
+      }
+      if constexpr (LAYOUT == TERN_Q2_0_G128) {
 #pragma unroll
-      for (int i = 0; i < C; i++) {
-        float tv;
-        if (LAYOUT == TERN_Q2_0_G128) {
-          const uint32_t f = (v >> (2 * i)) & 3u;  // two's complement field; 0b10 (invalid) reads as 0
-          tv = f == 1u ? 1.f : (f == 3u ? -1.f : 0.f);
-        } else if (LAYOUT == TERN_Q1_0_G128) {
-          tv = (v >> i) & 1u ? 1.f : -1.f;  // sign bit, 1 = +1
-        } else {
-          const uint32_t c = v % 3u;  // digit i, c = t + 1 (an invalid byte gives unspecified t)
-          v /= 3u;
-          tv = (float)((int)c - 1);
+        for (int c = 0; c < CL; c++) {  // field c % 16 of word c / 16 is column c
+          const float tv = __uint_as_float((w[c / 16] * (1u << (30 - 2 * (c % 16)))) & 0xC0000000u);
+#pragma unroll
+          for (int b = 0; b < B; b++) acc[c][b] = fmaf(tv, sd0[b], acc[c][b]);
         }
-        const float sc = (col0 + i) / kGroup == g_first ? s0 : s1;
+      } else if constexpr (LAYOUT == TERN_Q1_0_G128) {
 #pragma unroll
-        for (int b = 0; b < BATCH; b++) acc[i][b] = fmaf(tv, sc * d[b], acc[i][b]);
+        for (int c = 0; c < CL; c++) {  // bit c % 32 of word c / 32 is column c
+          const float tv = __uint_as_float(((w[c / 32] * (1u << (31 - (c % 32)))) & 0x80000000u) ^ 0xC0000000u);
+#pragma unroll
+          for (int b = 0; b < B; b++) acc[c][b] = fmaf(tv, sd0[b], acc[c][b]);
+        }
+      } else {
+#pragma unroll
+        for (int wd = 0; wd < NWD; wd++) {
+          uint32_t o[10];
+          dec_t3_word(w[wd], k0, o);
+#pragma unroll
+          for (int h = 0; h < 2; h++)
+#pragma unroll
+            for (int i = 0; i < 5; i++)
+#pragma unroll
+              for (int hi = 0; hi < 2; hi++) {
+                // byte h (low half) or 2 + h (high half) of the word, digit 4 - i
+                const int c = 5 * (4 * wd + h + 2 * hi) + (4 - i);
+                if (c < CL) {
+                  const float tv = __uint_as_float(hi ? (o[5 * h + i] & 0xC0000000u) : (o[5 * h + i] << 16));
+#pragma unroll
+                  for (int b = 0; b < B; b++) acc[c][b] = fmaf(tv, c < split ? sd0[b] : sd1[b], acc[c][b]);
+                }
+              }
+        }
       }
     }
   }
-  // sum the four row phases: phases 2, 3 hand their sums to phases 0, 1, which store theirs added
-  if (phase >= kPhases / 2) {
+  // sum the warps' row phases in warp order
+  float* mine = red + (size_t)warp * 32 * CL * B + (size_t)lane * CL * B;
 #pragma unroll
-    for (int i = 0; i < C; i++)
+  for (int c = 0; c < CL; c++)
 #pragma unroll
-      for (int b = 0; b < BATCH; b++) red[phase - kPhases / 2][byte * C + i][b] = acc[i][b];
-  }
+    for (int b = 0; b < B; b++) mine[c * B + b] = acc[c][b];
   __syncthreads();
-  if (phase < kPhases / 2) {
-#pragma unroll
-    for (int i = 0; i < C; i++)
-#pragma unroll
-      for (int b = 0; b < BATCH; b++) red[phase][byte * C + i][b] += acc[i][b];
-  }
-  __syncthreads();
-  for (int e = t; e < kTBytes * C * BATCH; e += kTThreads) {
-    const int c = e / BATCH, b = e % BATCH;
-    const int64_t col = (int64_t)blockIdx.x * kTBytes * C + c;
+  for (int e = threadIdx.x; e < 32 * CL * B; e += kTThreads) {
+    const int cl = e / B, b = e % B;
+    const int64_t col = (int64_t)blockIdx.x * 32 * CL + cl;
     if (b >= batch || col >= k) continue;
     float v = 0.f;
 #pragma unroll
-    for (int p = 0; p < kPhases / 2; p++) v += red[p][c][b];
+    for (int p = 0; p < kTWarps; p++) v += red[(size_t)p * 32 * CL * B + e];
     if (part) part[((int64_t)blockIdx.y * batch + b) * k + col] = v;
     else dx[(int64_t)b * k + col] = __half_as_ushort(__float2half_rn(v));
   }
@@ -109,14 +160,20 @@ __global__ void __launch_bounds__(256) gemv_t_reduce(const float* __restrict__ p
   }
 }
 
-template <int LAYOUT, int BATCH>
+int batch_slots(int64_t batch) { return batch <= 1 ? 1 : batch <= 2 ? 2 : batch <= 4 ? 4 : 8; }
+
+template <int LAYOUT, int B>
 cudaError_t launch_t(const tern_matrix& W, const uint16_t* dy, int batch, uint16_t* dx, float* part,
                      const GemvTPlan& p, cudaStream_t st) {
+  constexpr size_t smem = red_bytes<LAYOUT, B>();
+  auto kern = gemv_t_kernel<LAYOUT, B>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   dim3 grid(p.col_blocks, p.slices);
-  gemv_t_kernel<LAYOUT, BATCH><<<grid, kTThreads, 0, st>>>(static_cast<const uint8_t*>(W.codes), W.code_row_stride,
-                                                          W.scales, W.scale_row_stride, dy, batch, W.n, W.k,
-                                                          p.rows_per_slice, p.slices > 1 ? part : nullptr, dx);
-  cudaError_t e = cudaGetLastError();
+  kern<<<grid, kTThreads, smem, st>>>(static_cast<const uint8_t*>(W.codes), W.code_row_stride, W.scales,
+                                      W.scale_row_stride, dy, batch, W.n, W.k, row_bytes(W.layout, W.k),
+                                      p.rows_per_slice, p.slices > 1 ? part : nullptr, dx);
+  e = cudaGetLastError();
   if (e != cudaSuccess || p.slices == 1) return e;
   const int64_t total = (int64_t)batch * W.k;
   const int64_t blocks = (total + 255) / 256;
@@ -128,21 +185,25 @@ cudaError_t launch_t(const tern_matrix& W, const uint16_t* dy, int batch, uint16
 template <int LAYOUT>
 cudaError_t dispatch_t(const tern_matrix& W, const uint16_t* dy, int batch, uint16_t* dx, float* part,
                        const GemvTPlan& p, cudaStream_t st) {
-  if (batch <= 1) return launch_t<LAYOUT, 1>(W, dy, batch, dx, part, p, st);
-  if (batch <= 2) return launch_t<LAYOUT, 2>(W, dy, batch, dx, part, p, st);
-  if (batch <= 4) return launch_t<LAYOUT, 4>(W, dy, batch, dx, part, p, st);
-  return launch_t<LAYOUT, 8>(W, dy, batch, dx, part, p, st);
+  switch (batch_slots(batch)) {
+    case 1: return launch_t<LAYOUT, 1>(W, dy, batch, dx, part, p, st);
+    case 2: return launch_t<LAYOUT, 2>(W, dy, batch, dx, part, p, st);
+    case 4: return launch_t<LAYOUT, 4>(W, dy, batch, dx, part, p, st);
+    default: return launch_t<LAYOUT, 8>(W, dy, batch, dx, part, p, st);
+  }
 }
 
 }  // namespace
 
+// Column blocks of 32 lanes x LB bytes; row slices so that about two CTAs run per SM, each warp
+// reading at least 8 rows of its slice.
 GemvTPlan gemv_t_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
   GemvTPlan p{};
-  const int64_t cols = (int64_t)kTBytes * (layout == TERN_Q2_0_G128 ? 4 : layout == TERN_Q1_0_G128 ? 8 : 5);
-  p.col_blocks = (int)((k + cols - 1) / cols);
-  // about two CTAs per SM; every slice keeps at least 64 rows
+  const int64_t lb = (layout == TERN_Q1_0_G128 ? 8 : 16) / batch_slots(batch);
+  const int64_t block_bytes = 32 * lb;
+  p.col_blocks = (int)((row_bytes(layout, k) + block_bytes - 1) / block_bytes);
   int64_t slices = (2 * (int64_t)sms + p.col_blocks - 1) / p.col_blocks;
-  slices = std::max<int64_t>(1, std::min<int64_t>(slices, (n + 63) / 64));
+  slices = std::max<int64_t>(1, std::min<int64_t>(slices, (n + 8 * kTWarps - 1) / (8 * kTWarps)));
   p.rows_per_slice = (n + slices - 1) / slices;
   p.slices = (int)((n + p.rows_per_slice - 1) / p.rows_per_slice);
   p.ws_bytes = p.slices > 1 ? (size_t)p.slices * batch * k * sizeof(float) : 0;

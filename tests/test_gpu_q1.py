@@ -142,7 +142,7 @@ def test_gemv_closed_forms():
 
 
 def test_gemv_split_k_deterministic_and_workspace_reuse():
-    n, k, batch = 1000, 17408, 5  # three launches of the pair kernel share one workspace
+    n, k, batch = 1001, 17408, 5  # n % 8 != 0: three launches of the pair kernel share one workspace
     codes, s, x = workload(Q1, n, k, batch, seed=12)
     W = _matrix(codes, s, k)
     ws = T.gemv_workspace(W, batch)
