@@ -294,7 +294,7 @@ def run_native(args, rank, world, local_rank):
     ms = e0.elapsed_time(e1)
     ms = max_over_ranks(torch, ms, world, dev)
     ms_per_step = ms / args.steps
-    value = set_bytes * args.steps * world / (ms * 1e-3) / 1e9
+    value = replica_throughput(set_bytes, args.steps, world, ms)
 
     # per-kernel launch durations in the same steady state (events around single-kernel graphs)
     per_kernel = time_kernels(torch, T, W, xs, ys, wss, mats, copies, stream)
@@ -328,6 +328,21 @@ def run_native(args, rank, world, local_rank):
         if extras:
             line["rows"] = extras
         print(json.dumps(line), flush=True)
+
+
+def init_dist(world, local_rank, backend="nccl"):
+    """One process per GPU (nccl), or per CPU rank (gloo, for the host-side tests of this path); ranks
+    that wait for one another end with an error after two minutes."""
+    import datetime
+    import torch
+    if backend == "nccl":
+        torch.cuda.set_device(local_rank)
+    torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+
+
+def replica_throughput(bytes_per_step, steps, world, ms):
+    """Whole-job GB/s of `world` replicas that each ran `steps` steps, timed as the max over ranks."""
+    return bytes_per_step * steps * world / (ms * 1e-3) / 1e9
 
 
 def max_over_ranks(torch, v, world, dev):
@@ -663,10 +678,7 @@ def main():
         run_reference(args, rank, world)
         return
     if world > 1:
-        import datetime
-        import torch
-        torch.cuda.set_device(local_rank)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        init_dist(world, local_rank, "nccl")
     try:
         run_native(args, rank, world, local_rank)
     finally:
