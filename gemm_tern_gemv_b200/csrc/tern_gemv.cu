@@ -1,4 +1,4 @@
-// Decode GEMV y = W x for packed ternary W (batch 1..64) on mma.sync tensor cores.
+// Decode GEMV y = W x for packed ternary (and binary) W, batch 1..64, on mma.sync tensor cores.
 //
 // What is computed ("Ternary Bonsai 2 27B ..." discuss.pytorch.kr, section "그룹 단위 스케일을
 // 공유하는 삼진 형식", eq. w_i = s_g t_i; section "하이브리드 어텐션을 위한 저비트 커널": the
@@ -18,15 +18,19 @@
 //   * The 8 MMA columns carry (batch, group-within-window) pairs, so each group's partial sum gets
 //     its own scale in the fp32 epilogue. Activations are laid out once per CTA in fragment order.
 // Two kernels:
-//   * gemv_reg_kernel (Q2_0_g128 batch <= 4, base-3 batch <= 2): one window = 64 code bytes of each
-//     row of a 32-row warp tile; every warp streams its windows through its own ring of TMA boxes
-//     (codes and scales, out-of-range reads zero-filled) and decodes them in registers. The
-//     (tile, window) units of a K slice are split into equal runs, one per warp (stream-K), so every
-//     SM gets the same work whatever the matrix shape; tiles shared by several runs are summed
-//     deterministically by the last run to arrive.
+//   * gemv_reg_kernel (Q2_0_g128 batch <= 4, base-3 batch <= 2, binary Q1_0_g128 in pairs of batch
+//     rows): one window = 64 code bytes of each row of a 32-row warp tile; every warp streams its
+//     windows through its own ring of TMA boxes (codes and scales, out-of-range reads zero-filled) and
+//     decodes them in registers. Work split: when K is one slice, each CTA owns whole row tiles and its
+//     warps split them into equal runs, shared tiles being summed in shared memory (CTA-local);
+//     otherwise the (tile, window) units of a K slice are split into equal runs dealt over all warps
+//     (stream-K) and tiles shared by several runs are summed through the workspace by the last run to
+//     arrive. Both orders are deterministic. 16 warps x 1 CTA or 8 warps x 2 CTAs per SM, by the
+//     number of row tiles. As a programmatic dependent launch it can request its first weight boxes
+//     before the preceding kernel on the stream completes (see tern_gemv_ex).
 //   * gemv_kernel (larger batches): per-warp cp.async rings over 32- or 16-row tiles, base-3
 //     windows expanded to 2-bit fields in shared memory first; K is split across CTAs for narrow
-//     matrices, with the same last-arriver reduction.
+//     matrices, with the last-arriver reduction.
 #include <cuda_fp16.h>
 
 #include <algorithm>
