@@ -75,10 +75,6 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src, bool vali
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0)
                : "memory");
 }
-__device__ __forceinline__ void cp_async4(void* dst, const void* src, bool valid) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 4 : 0)
-               : "memory");
-}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
@@ -644,12 +640,6 @@ __host__ __device__ constexpr uint32_t s_stage_bytes(int layout, int rt) {
 __host__ __device__ inline size_t s_smem_bytes(int layout, int rt, int stages, int gps, int bs, int nw) {
   return (size_t)s_frag_window_bytes(layout, bs) * (s_windows(layout, gps) + 1) +
          (size_t)nw * stages * (s_stage_bytes(layout, rt) + 8) + 16;  // + full barriers, abort flag
-}
-
-__device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
-  int old;
-  asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
 }
 
 __device__ __forceinline__ uint32_t lds16(uint32_t addr) {
