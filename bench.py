@@ -308,7 +308,8 @@ def run_native(args, rank, world, local_rank):
                                for r in per_kernel]}
 
     e2e = measure_e2e(torch, T, W, mats, copies, args, stream, world, dev, set_bytes)
-    extras = {} if args.no_extras else measure_extras(torch, T, dev, peaks, stream)
+    # the other rows are single-GPU measurements: taken at N = 1 only, so scaling runs stay short
+    extras = {} if (args.no_extras or world > 1) else measure_extras(torch, T, dev, peaks, stream)
     cpu = cpu_baseline(torch, T, W, xs, mats) if (rank == 0 and world == 1) else None
 
     if rank == 0:
