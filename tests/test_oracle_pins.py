@@ -39,7 +39,7 @@ def _golden_hand():
                 continue
             lhs, rhs = line.split("->")
             parts = lhs.split()
-            layout = O.Q2_0_G128 if parts[0] == "Q2" else O.T3_5PB_G128
+            layout = {"Q2": O.Q2_0_G128, "T3": O.T3_5PB_G128, "Q1": O.Q1_0_G128}[parts[0]]
             t = [int(v) for v in parts[1:]]
             b = [int(v, 16) for v in rhs.split()]
             cases.append((layout, t, b))
@@ -112,12 +112,16 @@ def test_t3_byte_table_exhaustive():
 
 
 def test_hand_packed_golden():
+    seen = set()
     for layout, t, expect in _golden_hand():
-        row = np.zeros((1, 128), dtype=np.int8)
+        seen.add(layout)
+        # the rest of the row is t = 0 (t = -1 for the binary layout, which has no zero)
+        row = np.full((1, 128), -1 if layout == O.Q1_0_G128 else 0, dtype=np.int8)
         row[0, : len(t)] = t
         p = O.pack(row, layout)
         assert list(p[0, : len(expect)]) == expect, (layout, t)
         assert list(O.unpack(p, layout, 128)[0]) == list(row[0])
+    assert seen == set(O.LAYOUTS)
 
 
 def test_t3_padding_bytes():
