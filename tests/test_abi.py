@@ -214,3 +214,18 @@ def test_gemv_t_rejects_before_launch(lib):
     assert lib.tern_gemv_t(ctypes.byref(m), P(FAKE + 1), 1, P(FAKE), None, 0, None) == 3
     assert lib.tern_gemv_t(ctypes.byref(m), P(FAKE), 1, P(FAKE), None, 0, None) == 4
     assert lib.tern_gemv_t(ctypes.byref(m), P(FAKE), 1, P(FAKE), P(FAKE + 8), need, None) == 3
+
+
+def test_noalloc_scratch_claim_of_the_header(lib):
+    # tern.h: batch <= 8 fits the static scratch for N <= 151936 at K = 4096 and for N <= 34816 up to
+    # K = 17408 (the plan arithmetic is host-side, so the workspace size can be checked without a GPU)
+    limit = 8 << 20
+    for layout, rb in ((1, lambda k: k // 4), (2, lambda k: -(-(-(-k // 5)) // 16) * 16), (3, lambda k: k // 8)):
+        for b in (1, 2, 3, 4, 5, 8):
+            for n in (128, 4096, 24576, 65536, 151936):
+                m = _mat(layout=layout, n=n, k=4096, code_row_stride=rb(4096), scale_row_stride=32)
+                assert lib.tern_gemv_workspace_bytes(ctypes.byref(m), b) <= limit
+            for k in (1024, 5120, 12288, 17408):
+                for n in (1000, 5120, 34816):
+                    m = _mat(layout=layout, n=n, k=k, code_row_stride=rb(k), scale_row_stride=k // 128)
+                    assert lib.tern_gemv_workspace_bytes(ctypes.byref(m), b) <= limit
