@@ -35,6 +35,10 @@ class TernError(RuntimeError):
         super().__init__(f"{what}: {STATUS.get(status, status)} ({_status_string(status)})")
 
 
+class TernGemvOptsC(ctypes.Structure):
+    _fields_ = [("flags", ctypes.c_uint32), ("device_status", ctypes.c_void_p), ("wait_limit_ns", ctypes.c_uint64)]
+
+
 class TernMatrixC(ctypes.Structure):
     _fields_ = [("layout", ctypes.c_int32), ("n", ctypes.c_int64), ("k", ctypes.c_int64),
                 ("codes", ctypes.c_void_p), ("code_row_stride", ctypes.c_int64),
@@ -57,6 +61,8 @@ SIGNATURES = {
                                  ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "tern_gemv_ex": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                     ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint32, ctypes.c_void_p]),
+    "tern_gemv_opt": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                     ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(TernGemvOptsC), ctypes.c_void_p]),
     "tern_gemv_noalloc": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                          ctypes.c_void_p]),
     "tern_gemm": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
@@ -262,6 +268,29 @@ def gemv(W: TernMatrix, x, y=None, workspace=None, static_weights: bool = False)
     else:
         st = lib().tern_gemv(ctypes.byref(c), _ptr(x), batch, _ptr(y), _ptr(workspace), wsb, _stream_handle())
         _check(st, "tern_gemv")
+    return y
+
+
+def gemv_opt(W: TernMatrix, x, y=None, workspace=None, static_weights: bool = False, status=None,
+             wait_limit_ns: int = 0):
+    """tern_gemv_opt: gemv with an optional device status word (uint32 tensor, TERN_DEVICE_TIMEOUT is
+    OR-ed in when a pipeline wait runs out) and a bound on each wait (0 = the library default)."""
+    torch = _torch()
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    batch = x.shape[0]
+    x = x.contiguous()
+    if y is None:
+        y = torch.empty((batch, W.n), dtype=torch.float16, device=x.device)
+    if workspace is None:
+        workspace = gemv_workspace(W, batch)
+    wsb = workspace.numel() if workspace is not None else 0
+    c = W.c()
+    o = TernGemvOptsC(GEMV_STATIC_WEIGHTS if static_weights else 0, _ptr(status) if status is not None else None,
+                      int(wait_limit_ns))
+    st = lib().tern_gemv_opt(ctypes.byref(c), _ptr(x), batch, _ptr(y), _ptr(workspace), wsb, ctypes.byref(o),
+                             _stream_handle())
+    _check(st, "tern_gemv_opt")
     return y
 
 

@@ -21,7 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libtern.so")
 
-SOURCES = ["tern_api.cu", "tern_pack.cu", "tern_gemv.cu", "tern_gemm.cu", "tern_tmap.cu", "tern_rotate.cu", "tern_gemv_t.cu"]
+SOURCES = ["tern_api.cu", "tern_pack.cu", "tern_gemv.cu", "tern_gemv_i8.cu", "tern_gemm.cu", "tern_tmap.cu", "tern_rotate.cu", "tern_gemv_t.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I" + INCLUDE, "-I" + CSRC]

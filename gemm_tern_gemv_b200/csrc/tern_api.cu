@@ -141,7 +141,18 @@ tern_status tern_gemv(const tern_matrix* W, const uint16_t* x, int64_t batch, ui
 
 tern_status tern_gemv_ex(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y, void* workspace,
                          size_t workspace_bytes, uint32_t flags, void* stream) {
+  tern_gemv_opts o{};
+  o.flags = flags;
+  return tern_gemv_opt(W, x, batch, y, workspace, workspace_bytes, &o, stream);
+}
+
+tern_status tern_gemv_opt(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y, void* workspace,
+                          size_t workspace_bytes, const tern_gemv_opts* opts, void* stream) {
+  const uint32_t flags = opts ? opts->flags : 0u;
+  uint32_t* status = opts ? opts->device_status : nullptr;
+  const uint64_t wait_ns = opts ? opts->wait_limit_ns : 0u;
   if (flags & ~(uint32_t)TERN_GEMV_STATIC_WEIGHTS) return TERN_ERR_INVALID_ARG;
+  if (status && (reinterpret_cast<uintptr_t>(status) & 3u)) return TERN_ERR_ALIGNMENT;
   tern_status s = check_matrix(W);
   if (s != TERN_OK) return s;
   if (batch < 1 || batch > TERN_GEMV_MAX_BATCH || !x || !y) return TERN_ERR_INVALID_ARG;
@@ -152,7 +163,8 @@ tern_status tern_gemv_ex(const tern_matrix* W, const uint16_t* x, int64_t batch,
     if (!workspace || workspace_bytes < plan.ws_bytes) return TERN_ERR_WORKSPACE;
     if (!aligned16(workspace)) return TERN_ERR_ALIGNMENT;
   }
-  return from_cuda(launch_gemv(*W, x, (int)batch, y, workspace, plan, static_cast<cudaStream_t>(stream), flags));
+  return from_cuda(launch_gemv(*W, x, (int)batch, y, workspace, plan, static_cast<cudaStream_t>(stream), flags,
+                               status, wait_ns));
 }
 
 tern_status tern_gemv_noalloc(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y, void* stream) {

@@ -68,6 +68,8 @@ struct Args {
   uint32_t unit;    // always 1 (see `mul` in the kernel)
   int early;        // register kernel: W may be read before earlier work on the stream completes
   int local;        // register kernel: CTA-local reduction of whole tiles (no workspace)
+  uint32_t* status;  // register kernel: optional device status word (TERN_DEVICE_TIMEOUT on a wait that ran out)
+  uint64_t wait_ns;  // register kernel: bound on each pipeline wait
 };
 
 // ---- small device helpers --------------------------------------------------------------------
@@ -957,7 +959,9 @@ __global__ void __launch_bounds__(NW * 32, CPS)
   bool has_first = false;
   int st = 0;
   for (; st < total; st++) {
-    if (!sm100::mbar_wait_bounded(full + c_slot, (st / STAGES) & 1, abort_flag, nullptr, 0u, kRegWaitLimitNs)) break;
+    if (!sm100::mbar_wait_bounded(full + c_slot, (st / STAGES) & 1, abort_flag, a.status, TERN_DEVICE_TIMEOUT,
+                                  a.wait_ns))
+      break;
     const uint32_t stage_u = ring_u + c_slot * STAGE;
     // codes of the window; activation fragments follow one code word ahead of the MMAs that use them
     // (fewer live registers than a whole window's worth, latency still covered)
@@ -1392,6 +1396,18 @@ bool gemv_supported(int32_t layout, int64_t n, int64_t k, int64_t batch) {
 }
 
 GemvPlan gemv_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
+  // batches 1-2 on the int8-plane kernel; binary batches the GEMM does not take as pairs of rows on it
+  const bool bin_pairs = layout == TERN_Q1_0_G128 && !use_gemm(layout, n, batch);
+  if (batch <= 2 || bin_pairs) {
+    const I8Plan ip = i8_plan(layout, n, k, std::min<int64_t>(batch, 2), sms);
+    if (ip.ok) {
+      GemvPlan p{};
+      p.i8 = true;
+      p.i8p = ip;
+      p.splits = 1;
+      return p;
+    }
+  }
   if (use_gemm(layout, n, batch)) {
     GemvPlan p{};
     p.gemm = true;
@@ -1425,8 +1441,17 @@ GemvPlan gemv_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms)
 }
 
 cudaError_t launch_gemv(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y, void* workspace,
-                        const GemvPlan& plan, cudaStream_t st, uint32_t flags) {
-  if (plan.gemm) return launch_gemm(W, x, batch, y, nullptr, st);
+                        const GemvPlan& plan, cudaStream_t st, uint32_t flags, uint32_t* status, uint64_t wait_ns) {
+  if (plan.i8) {
+    // one launch per pair of rows of x, in order on the stream (binary batches 3-4)
+    for (int b0 = 0; b0 < batch; b0 += 2) {
+      const cudaError_t e = launch_gemv_i8(W, x + (int64_t)b0 * W.k, std::min(2, batch - b0), y + (int64_t)b0 * W.n,
+                                           plan.i8p, st, flags, status, wait_ns);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
+  if (plan.gemm) return launch_gemm(W, x, batch, y, status, st);
   Args a;
   a.codes = static_cast<const uint8_t*>(W.codes);
   a.cstride = W.code_row_stride;
@@ -1446,6 +1471,8 @@ cudaError_t launch_gemv(const tern_matrix& W, const uint16_t* x, int batch, uint
   a.kmax = plan.kmax;
   a.early = (flags & TERN_GEMV_STATIC_WEIGHTS) ? 1 : 0;
   a.local = plan.local ? 1 : 0;
+  a.status = status;
+  a.wait_ns = wait_ns ? wait_ns : kRegWaitLimitNs;
   a.ws = plan.ws_bytes ? static_cast<float*>(workspace) : nullptr;
   a.counters = plan.ws_bytes ? reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + plan.ws_partial_bytes) : nullptr;
   if (plan.reg && W.layout == TERN_Q1_0_G128) {

@@ -34,6 +34,24 @@ cudaError_t launch_pack(int32_t layout, int64_t n, int64_t k, const uint16_t* w,
 cudaError_t launch_unpack(const tern_matrix& W, uint16_t* w_out, int64_t w_stride, int8_t* t_out,
                           int64_t t_stride, int32_t* invalid_count, cudaStream_t st);
 
+// Plan of the int8-plane GEMV (batch 1-2): K slices per cluster, consumer warps, TMA stage geometry.
+struct I8Plan {
+  bool ok;
+  int ks;          // K slices = CTAs per cluster (1, 2 or 4)
+  int L;           // units per slice
+  int nw;          // consumer warps per CTA
+  int npr;         // 1: each consumer warp owns exactly one unit of a slice
+  int units, tiles, groups;
+  int box_b, nfull, rem_b, sc_w;  // TMA boxes of one stage
+  int code_bytes, stage_bytes, stages;
+  int xk;          // activations per CTA (halves)
+  int tmax;        // tiles per cluster (upper bound)
+};
+I8Plan i8_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms);
+// status / wait_ns: optional device status word and bound on each pipeline wait (0 = 1 s)
+cudaError_t launch_gemv_i8(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y, const I8Plan& pl,
+                           cudaStream_t st, uint32_t flags, uint32_t* status, uint64_t wait_ns);
+
 // Split-K plan of the decode GEMV for one (layout, n, k, batch) on a device with `sms` SMs.
 struct GemvPlan {
   bool gemm;            // Q2_0_g128 with many rows of x: the tcgen05 GEMM kernel (no workspace)
@@ -49,6 +67,8 @@ struct GemvPlan {
   int warps;            // register kernel: warps per CTA (16, one CTA per SM; or 8, two per SM)
   size_t ws_partial_bytes;  // fp32 partial sums [splits * slots][batch][n]
   size_t ws_bytes;          // partials + one int32 counter per row block, rounded to 16
+  bool i8;                  // batch 1-2: the int8-plane kernel (no workspace)
+  I8Plan i8p;
 };
 GemvPlan gemv_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms);
 // False only for a binary matrix too large for the register kernel's 32-bit unit indices at a batch
@@ -56,8 +76,10 @@ GemvPlan gemv_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms)
 bool gemv_supported(int32_t layout, int64_t n, int64_t k, int64_t batch);
 
 // flags: TERN_GEMV_* bits of tern_gemv_ex (0 for tern_gemv).
+// status / wait_ns: optional device status word and wait bound of the kernels that wait on a pipeline.
 cudaError_t launch_gemv(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y,
-                        void* workspace, const GemvPlan& plan, cudaStream_t st, uint32_t flags = 0);
+                        void* workspace, const GemvPlan& plan, cudaStream_t st, uint32_t flags = 0,
+                        uint32_t* status = nullptr, uint64_t wait_ns = 0);
 
 // tern_gemv_noalloc's work after argument checks (scratch in a static device array).
 tern_status gemv_noalloc(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y, cudaStream_t st);

@@ -196,6 +196,25 @@ TERN_API tern_status tern_gemv(const tern_matrix* W, const uint16_t* x, int64_t 
 TERN_API tern_status tern_gemv_ex(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y,
                                   void* workspace, size_t workspace_bytes, uint32_t flags, void* stream);
 
+/* Options of tern_gemv_opt. Zero-initialise and set what you need. */
+typedef struct tern_gemv_opts {
+  uint32_t flags;            /* 0 or TERN_GEMV_STATIC_WEIGHTS (see tern_gemv_ex) */
+  uint32_t* device_status;   /* device uint32 or NULL: TERN_DEVICE_TIMEOUT is OR-ed in when a pipeline
+                                wait of the call runs out; the caller zeroes it and reads it back */
+  uint64_t wait_limit_ns;    /* bound on each internal pipeline wait; 0 = the default of one second */
+} tern_gemv_opts;
+
+/* tern_gemv_ex with a device status word and a wait bound. The pages ask a runtime to refuse loudly
+ * what it cannot carry out rather than emit garbage ("Ternary Bonsai 2 27B ..." discuss.pytorch.kr,
+ * the runtime notes after section "블록 단위 하다마드 회전"); a GEMV whose pipeline wait runs out
+ * (a producer that never delivers, a limit set too short) abandons its tiles, writes NaN to the
+ * outputs of the rows it owns (batches 1-2), and reports TERN_DEVICE_TIMEOUT through device_status.
+ * It never traps or hangs. Same arguments, result and errors as tern_gemv_ex otherwise, plus
+ * TERN_ERR_ALIGNMENT for a device_status that is not 4-byte aligned. opts may be NULL (= all zero). */
+TERN_API tern_status tern_gemv_opt(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y,
+                                   void* workspace, size_t workspace_bytes, const tern_gemv_opts* opts,
+                                   void* stream);
+
 /* Bytes of device memory tern_gemv_noalloc keeps for its split-K scratch (per GPU, for the
  * lifetime of the process). */
 #define TERN_GEMV_NOALLOC_SCRATCH_BYTES (8u << 20)

@@ -97,9 +97,10 @@ def test_gemv_ex_rejects_unknown_flags(lib):
     args = (ctypes.byref(m), ctypes.c_void_p(FAKE), 1, ctypes.c_void_p(FAKE), None, 0)
     assert lib.tern_gemv_ex(*args, 2, None) == 1
     assert lib.tern_gemv_ex(*args, 0x80000000, None) == 1
-    # a valid flag passes the flag check and stops at the next host-side check (missing workspace)
+    # a valid flag passes the flag check and stops at the next host-side check (missing workspace;
+    # batch 4 of this shape runs split-K)
     w = _mat(n=5120, k=17408, code_row_stride=4352, scale_row_stride=136)
-    assert lib.tern_gemv_ex(ctypes.byref(w), ctypes.c_void_p(FAKE), 1, ctypes.c_void_p(FAKE), None, 0, 1, None) == 4
+    assert lib.tern_gemv_ex(ctypes.byref(w), ctypes.c_void_p(FAKE), 4, ctypes.c_void_p(FAKE), None, 0, 1, None) == 4
 
 
 def test_gemv_rejects_bad_batch_and_buffers(lib):
@@ -112,15 +113,21 @@ def test_gemv_rejects_bad_batch_and_buffers(lib):
 
 
 def test_gemv_workspace_size_and_rejection(lib):
-    # a narrow matrix with a long K needs split-K workspace; too little is refused before any launch
+    # a narrow matrix with a long K at batch 4 needs split-K workspace; too little is refused before
+    # any launch
     m = _mat(n=5120, k=17408, code_row_stride=4352, scale_row_stride=136)
-    need = lib.tern_gemv_workspace_bytes(ctypes.byref(m), 1)
+    need = lib.tern_gemv_workspace_bytes(ctypes.byref(m), 4)
     assert need > 0 and need % 16 == 0
-    assert lib.tern_gemv(ctypes.byref(m), ctypes.c_void_p(FAKE), 1, ctypes.c_void_p(FAKE), None, 0, None) == 4
-    assert lib.tern_gemv(ctypes.byref(m), ctypes.c_void_p(FAKE), 1, ctypes.c_void_p(FAKE),
+    assert lib.tern_gemv(ctypes.byref(m), ctypes.c_void_p(FAKE), 4, ctypes.c_void_p(FAKE), None, 0, None) == 4
+    assert lib.tern_gemv(ctypes.byref(m), ctypes.c_void_p(FAKE), 4, ctypes.c_void_p(FAKE),
                          ctypes.c_void_p(FAKE), need - 16, None) == 4
-    assert lib.tern_gemv(ctypes.byref(m), ctypes.c_void_p(FAKE), 1, ctypes.c_void_p(FAKE),
+    assert lib.tern_gemv(ctypes.byref(m), ctypes.c_void_p(FAKE), 4, ctypes.c_void_p(FAKE),
                          ctypes.c_void_p(FAKE + 8), need, None) == 3
+    # batches 1 and 2 split K over thread-block clusters instead and need none, in every layout
+    for layout, rb in ((1, 4352), (2, 3488), (3, 2176)):
+        w = _mat(layout=layout, n=5120, k=17408, code_row_stride=rb, scale_row_stride=136)
+        assert lib.tern_gemv_workspace_bytes(ctypes.byref(w), 1) == 0
+        assert lib.tern_gemv_workspace_bytes(ctypes.byref(w), 2) == 0
     # a matrix of one 128-weight group per row is never split and needs none; neither do the 8B-class
     # decode shapes at batch 1, whose tiles are summed inside each CTA
     one = _mat(n=4096, k=128, code_row_stride=32, scale_row_stride=8)
@@ -138,13 +145,16 @@ def test_gemv_workspace_size_and_rejection(lib):
 
 
 def test_binary_gemv_workspace_is_that_of_two_rows(lib):
-    # the binary register kernel runs batch rows in pairs, one launch after another on the stream,
-    # so every batch below the GEMM's reuses the workspace of a two-row launch
+    # binary batches below the GEMM's run as pairs of rows, one launch after another on the stream,
+    # so every such batch reuses the workspace of a two-row launch (none on the int8-plane kernel;
+    # K = 17280 is not a multiple of 256 and runs on the register kernel, which needs one)
+    for k, rb, need in ((17408, 2176, False), (17280, 2160, True)):
+        m = _mat(layout=3, n=5120, k=k, code_row_stride=rb, scale_row_stride=k // 128 + 7 & ~7)
+        two = lib.tern_gemv_workspace_bytes(ctypes.byref(m), 2)
+        assert (two > 0) == need
+        for b in (3, 4):
+            assert lib.tern_gemv_workspace_bytes(ctypes.byref(m), b) == two
     m = _mat(layout=3, n=5120, k=17408, code_row_stride=2176, scale_row_stride=136)
-    two = lib.tern_gemv_workspace_bytes(ctypes.byref(m), 2)
-    assert two > 0
-    for b in (3, 4):
-        assert lib.tern_gemv_workspace_bytes(ctypes.byref(m), b) == two
     for b in (5, 16, 17):  # the GEMM kernel takes binary batches from 5 on (n % 8 == 0)
         assert lib.tern_gemv_workspace_bytes(ctypes.byref(m), b) == 0
     odd = _mat(layout=3, n=5121, k=17408, code_row_stride=2176, scale_row_stride=136)
@@ -221,11 +231,11 @@ def test_noalloc_scratch_claim_of_the_header(lib):
     # K = 17408 (the plan arithmetic is host-side, so the workspace size can be checked without a GPU)
     limit = 8 << 20
     for layout, rb in ((1, lambda k: k // 4), (2, lambda k: -(-(-(-k // 5)) // 16) * 16), (3, lambda k: k // 8)):
-        for b in (1, 2, 3, 4, 5, 8):
+        for b in range(1, 9):
             for n in (128, 4096, 24576, 65536, 151936):
                 m = _mat(layout=layout, n=n, k=4096, code_row_stride=rb(4096), scale_row_stride=32)
                 assert lib.tern_gemv_workspace_bytes(ctypes.byref(m), b) <= limit
             for k in (1024, 5120, 12288, 17408):
-                for n in (1000, 5120, 34816):
+                for n in (1000, 5120, 34816, 151936 if k == 4096 else 34816):
                     m = _mat(layout=layout, n=n, k=k, code_row_stride=rb(k), scale_row_stride=k // 128)
                     assert lib.tern_gemv_workspace_bytes(ctypes.byref(m), b) <= limit

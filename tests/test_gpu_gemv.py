@@ -80,7 +80,7 @@ def test_activation_dynamic_range():
 
 @pytest.mark.parametrize("layout", LAYOUTS)
 def test_split_k_deterministic_and_workspace_reuse(layout):
-    n, k, batch = 1000, 17408, 2
+    n, k, batch = 1000, 17408, 4
     codes, s, x = workload(layout, n, k, batch, seed=11)
     W = T.from_packed(torch.from_numpy(codes).cuda(), torch.from_numpy(s).cuda(), layout, k)
     ws = T.gemv_workspace(W, batch)
@@ -94,6 +94,24 @@ def test_split_k_deterministic_and_workspace_reuse(layout):
     rows = sample_rows(n, 256, 1)
     y_ref, a = O.gemv(codes, s, x, layout, k, rows=rows)
     check_product(y1.cpu().numpy()[:, rows], y_ref, a, "split-K")
+
+
+@pytest.mark.parametrize("layout", LAYOUTS + [T.Q1_0_G128])
+@pytest.mark.parametrize("n,k,batch", [(1000, 17408, 1), (1000, 17408, 2), (5120, 17408, 1), (300, 5120, 2)])
+def test_cluster_k_split_is_deterministic(layout, n, k, batch):
+    # batches 1-2 of narrow matrices split K over a thread-block cluster and add the slices through
+    # distributed shared memory in a fixed order: no workspace, and repeated calls agree bit for bit
+    codes, s, x = workload(layout, n, k, batch, seed=n + k + 17)
+    W = T.from_packed(torch.from_numpy(codes).cuda(), torch.from_numpy(s).cuda(), layout, k)
+    assert T.gemv_workspace(W, batch) is None
+    xg = torch.from_numpy(x).cuda()
+    y1 = T.gemv(W, xg).clone()
+    y2 = T.gemv(W, xg, static_weights=True).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    rows = sample_rows(n, 384, 7)
+    y_ref, a = O.gemv(codes, s, x, layout, k, rows=rows)
+    check_product(y1.cpu().numpy()[:, rows], y_ref, a, "cluster K split")
 
 
 @pytest.mark.parametrize("layout", LAYOUTS)

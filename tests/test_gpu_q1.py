@@ -141,12 +141,16 @@ def test_gemv_closed_forms():
         check_product(y, sign * (gs @ s.astype(np.float64).T), a, f"all {sign:+d}")
 
 
-def test_gemv_split_k_deterministic_and_workspace_reuse():
-    n, k, batch = 1001, 17408, 5  # n % 8 != 0: three launches of the pair kernel share one workspace
+@pytest.mark.parametrize("k,needs_ws", [(17408, False), (17280, True)])
+def test_gemv_split_k_deterministic_and_workspace_reuse(k, needs_ws):
+    # n % 8 != 0 keeps batch 5 off the GEMM: three launches of a two-row kernel, one after another.
+    # K = 17408 runs them on the int8-plane kernel (K split over a cluster, no workspace); K = 17280
+    # (not a multiple of 256) on the register kernel, whose three launches share one workspace.
+    n, batch = 1001, 5
     codes, s, x = workload(Q1, n, k, batch, seed=12)
     W = _matrix(codes, s, k)
     ws = T.gemv_workspace(W, batch)
-    assert ws is not None
+    assert (ws is not None) == needs_ws
     xg = torch.from_numpy(x).cuda()
     y1 = T.gemv(W, xg, workspace=ws).clone()
     y2 = T.gemv(W, xg, workspace=ws).clone()

@@ -28,20 +28,20 @@ def _noalloc(W, x, y):
 
 
 @pytest.mark.parametrize("layout", [T.Q2_0_G128, T.T3_5PB_G128, T.Q1_0_G128])
-@pytest.mark.parametrize("n,k,batch", [(4096, 4096, 1), (5120, 17408, 1), (1000, 2176, 3), (4096, 12288, 8),
+@pytest.mark.parametrize("n,k,batch", [(4096, 4096, 1), (5120, 17408, 4), (1000, 2176, 3), (4096, 12288, 8),
                                        (24576, 4096, 1), (300, 640, 2)])
 def test_noalloc_matches_gemv_twice(layout, n, k, batch):
     codes, s, x = workload(layout, n, k, batch, seed=n + k + batch)
     W = T.from_packed(torch.from_numpy(codes).cuda(), torch.from_numpy(s).cuda(), layout, k)
     xg = torch.from_numpy(x).cuda()
-    ref = T.gemv(W, xg).cpu().numpy().astype(np.float64)
-    _, a = O.gemv(codes, s, x, layout, k)  # sum_k |w_k x_k| of every output: the tolerance scale
+    y_ref, a = O.gemv(codes, s, x, layout, k)  # the fp64 oracle and sum_k |w_k x_k| of every output
+    ref = T.gemv(W, xg)
     for _ in range(2):  # two calls in a row: the shared scratch must be reusable
         y = torch.full((batch, n), float("nan"), dtype=torch.float16, device="cuda")
         assert _noalloc(W, xg, y) == 0
         torch.cuda.synchronize()
-        got = y.cpu().numpy().astype(np.float64)
-        check_product(got, ref, a, f"noalloc layout {layout} {n}x{k} b{batch}")
+        check_product(y.cpu().numpy().astype(np.float64), y_ref, a, f"noalloc layout {layout} {n}x{k} b{batch}")
+        assert torch.equal(y, ref)  # and the same bits as the workspace entry point
 
 
 def test_noalloc_rejects_oversized_scratch():
@@ -56,13 +56,18 @@ def test_noalloc_rejects_oversized_scratch():
 
 
 def test_noalloc_binding_roundtrip():
-    n, k = 2048, 4096
+    # a shape whose plan uses split-K scratch, so the binding reaches the static array
+    n, k, batch = 5120, 17408, 4
     t = synth.ternary_codes(n, k, seed=3)
     s = synth.group_scales(n, k // 128, seed=3)
-    x = synth.activations(1, k, seed=3)
+    x = synth.activations(batch, k, seed=3)
     W = T.from_packed(torch.from_numpy(pack_rows(t, T.Q2_0_G128)).cuda(), torch.from_numpy(s).cuda(), T.Q2_0_G128, k)
+    assert T.gemv_workspace_bytes(W, batch) > 0
     xg = torch.from_numpy(x).cuda()
     y1 = T.gemv_noalloc(W, xg)
     y2 = T.gemv(W, xg)
     torch.cuda.synchronize()
     assert torch.equal(y1, y2)  # same kernel and plan: identical bits
+    rows = np.arange(0, n, 7)
+    y_ref, a = O.gemv(pack_rows(t, T.Q2_0_G128), s, x, T.Q2_0_G128, k, rows=rows)
+    check_product(y1.cpu().numpy()[:, rows], y_ref, a, "noalloc binding")
