@@ -2,8 +2,9 @@
 
 Workload (one "step"): the 8B-class decode layer set at batch 1 in both packed layouts — GEMVs
 N x K = 4096 x 4096 (attention projection), 24576 x 4096 (fused gate/up), 4096 x 12288 (down),
-each in Q2_0_g128 and in base-3 (5 trits/byte) — i.e. six tern_gemv calls per step. Inputs are
-seeded synthetic codes (P(0)=0.4, P(+-1)=0.3), scales fp16(|N(0,1)|*0.02), activations fp16(N(0,1)).
+each in Q2_0_g128 and in base-3 (5 trits/byte) — and the LM head 151936 x 4096 in base-3 at batch 1,
+i.e. seven tern_gemv calls per step. Inputs are seeded synthetic codes (P(0)=0.4, P(+-1)=0.3), scales
+fp16(|N(0,1)|*0.02), activations fp16(N(0,1)).
 Metric: algorithmic bytes (packed codes + fp16 scales + x + y) per second, GB/s, whole job.
 
 L2 policy: the step rotates over enough copies of the weights that the footprint exceeds 3x the
@@ -32,10 +33,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 LAYER_SET = [(4096, 4096), (24576, 4096), (4096, 12288)]  # (N, K) of the 8B-class decode layers
+LM_HEAD = (151936, 4096)  # (N, K) of the LM head (base-3 layout)
 GROUP = 128
 L2_BYTES_DEFAULT = 126 * 1024 * 1024
 METRIC = "ternary GEMV GB/s (weights/s) & % of 8 TB/s HBM; GEMM TFLOP/s vs fp16 peak"
-WORKLOAD = "8B-class decode layer set, batch 1, Q2_0_g128 + base-3: 4096x4096, 24576x4096, 4096x12288"
+WORKLOAD = ("8B-class decode layer set (Q2_0_g128 + base-3: 4096x4096, 24576x4096, 4096x12288) and the "
+            "LM head 151936x4096 (base-3), batch 1")
 
 
 def _env_int(name, default):
@@ -54,7 +57,11 @@ def parse():
     p.add_argument("--no-extras", action="store_true", help="skip the per-row measurements of the other kernels")
     p.add_argument("--profile", default=None, metavar="CASE",
                    help="run a few launches of one kernel case for ncu: gemv_{q2|t3|q1}_NxK_bB, "
-                        "gemm_{q2|t3|q1}_MxNxK, pack_{q2|t3|q1}_NxK")
+                        "gemm_{q2|t3|q1}_MxNxK, pack_{q2|t3|q1}_NxK, unpack_{q2|t3|q1}_NxK, "
+                        "gemvt_{q2|t3|q1}_NxK_bB, rotate_bB_kK; or 'all' for one case of every kernel")
+    p.add_argument("--record-traffic", default=None, metavar="NCU_CSV",
+                   help="write profiles/traffic.json from an ncu --csv capture of the dominant GEMV "
+                        "(dram__bytes_read.sum + dram__bytes_write.sum), keyed by the current source digest")
     return p.parse_args()
 
 
@@ -116,6 +123,7 @@ class ClockSampler:
         self.stop = threading.Event()
         self.source = None
         self.t0 = self.t1 = None
+        self._sample = None
 
     def __enter__(self):
         try:
@@ -135,16 +143,21 @@ class ClockSampler:
                     "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
             mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
 
+            def one():
+                try:
+                    sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                    pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.rows.append((time.time(), sm, mx, pw, [k for k, b in bits.items() if r & b]))
+                except Exception:
+                    pass
+
             def poll():
                 while not self.stop.is_set():
-                    try:
-                        sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
-                        pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
-                        r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-                        self.rows.append((time.time(), sm, mx, pw, [k for k, b in bits.items() if r & b]))
-                    except Exception:
-                        pass
+                    one()
                     time.sleep(0.002)
+
+            self._sample = one
 
             self.thread = threading.Thread(target=poll, daemon=True)
             self.thread.start()
@@ -177,6 +190,11 @@ class ClockSampler:
             if len(parts) >= 9:
                 names = [self.NAMES[i] for i in range(4) if parts[5 + i].lower() == "active"]
                 self.rows.append((time.time(), num(parts[1]), num(parts[2]), num(parts[3]), names))
+
+    def sample_now(self):
+        """One synchronous sample (NVML only), taken while the GPU runs the timed work."""
+        if self._sample is not None:
+            self._sample()
 
     def begin(self):
         self.t0 = time.time()
@@ -234,7 +252,7 @@ def run_native(args, rank, world, local_rank):
     l2 = getattr(props, "L2_cache_size", L2_BYTES_DEFAULT) or L2_BYTES_DEFAULT
 
     layouts = [T.Q2_0_G128, T.T3_5PB_G128]
-    mats = [(layout, n, k) for layout in layouts for (n, k) in LAYER_SET]
+    mats = [(layout, n, k) for layout in layouts for (n, k) in LAYER_SET] + [(T.T3_5PB_G128,) + LM_HEAD]
     set_bytes = sum(algorithmic_bytes(l, n, k, 1) for (l, n, k) in mats)
     weight_bytes = sum(n * T.row_bytes(l, k) + n * (k // GROUP) * 2 for (l, n, k) in mats)
     copies = max(2, math.ceil(3 * l2 / weight_bytes))
@@ -288,6 +306,7 @@ def run_native(args, rank, world, local_rank):
             for i in range(args.steps):
                 graphs[i % copies].replay()
             e1.record(stream)
+            clk.sample_now()  # one sample while the queued replays run, however short the region
         e1.synchronize()
         clk.end()
     barrier()
@@ -318,6 +337,7 @@ def run_native(args, rank, world, local_rank):
                 "scaling": "weak", "vs_baseline": None, "dtype": "f16 (ternary codes, fp32 accumulate)",
                 "data": "synthetic (seeded codes P(0)=0.4, scales |N(0,1)|*0.02 fp16, x N(0,1) fp16)",
                 "config": {"workload": WORKLOAD, "batch": 1, "layouts": ["Q2_0_g128", "T3_5PB_g128"],
+                           "gemvs": [f"{'q2' if l == T.Q2_0_G128 else 't3'}_{n}x{k}" for (l, n, k) in mats],
                            "gemvs_per_step": launches_per_step, "bytes_per_step": set_bytes,
                            "l2": f"rotating {copies} weight copies ({copies * weight_bytes / 1e6:.0f} MB > 3x L2 "
                                  f"{l2 / 1e6:.0f} MB)", "parallelism": f"replicas x{world}",
@@ -436,7 +456,7 @@ def measure_e2e(torch, T, W, mats, copies, args, stream, world, dev, set_bytes):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms / steps, 6),
             "path": "C ABI tern_gemv_ex (TERN_GEMV_STATIC_WEIGHTS) via ctypes, eager launches; one pinned H2D "
-                    "of the six activation vectors and one D2H of the six results per step"}
+                    "of the step's activation vectors and one D2H of its results per step"}
 
 
 def measure_extras(torch, T, dev, peaks, stream):
@@ -573,8 +593,34 @@ def measure_extras(torch, T, dev, peaks, stream):
     return res
 
 
-def cpu_baseline(torch, T, W, xs, mats, rows=1024):
-    """The oracle, as it stands, on a bounded sample: `rows` rows of each of the six GEMVs."""
+def host_cpu():
+    """(logical CPUs, model name) of the host, as `nproc` and `lscpu` report them."""
+    n = os.cpu_count() or 1
+    model = None
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for line in out.splitlines():
+            if line.lower().startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except Exception:
+        pass
+    if model is None:
+        try:
+            with open("/proc/cpuinfo") as f:
+                for line in f:
+                    if line.startswith("model name"):
+                        model = line.split(":", 1)[1].strip()
+                        break
+        except Exception:
+            model = "unknown"
+    return n, model
+
+
+def cpu_baseline(torch, T, W, xs, mats, rows=1024, seconds=8.0):
+    """The oracle, as it stands, on a bounded sample (`rows` rows of each GEMV of the step), timed on
+    one thread and on all of the host's cores (numpy's BLAS threads); the all-cores figure is the
+    reported value."""
     import numpy as np
     import oracle as O
     try:
@@ -591,20 +637,67 @@ def cpu_baseline(torch, T, W, xs, mats, rows=1024):
         x = xs[i].cpu().numpy()
         samples.append((codes, sc, x, layout, k))
         nbytes += algorithmic_bytes(layout, len(r), k, 1)
-    ctx = threadpool_limits(limits=1) if threadpool_limits else None
-    t0 = time.perf_counter()
-    reps = 0
-    while True:
-        for (codes, sc, x, layout, k) in samples:
-            O.gemv(codes, sc, x, layout, k)
-        reps += 1
-        if time.perf_counter() - t0 > 10.0 or reps >= 50:
-            break
-    dt = time.perf_counter() - t0
-    if ctx is not None:
-        ctx.unregister() if hasattr(ctx, "unregister") else None
-    return {"value": round(nbytes * reps / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"first {rows} rows of each of the six GEMVs x {reps} passes ({dt:.1f} s, numpy fp64, 1 thread)"}
+
+    def leg(threads):
+        ctx = threadpool_limits(limits=threads) if threadpool_limits else None
+        t0 = time.perf_counter()
+        reps = 0
+        while True:
+            for (codes, sc, x, layout, k) in samples:
+                O.gemv(codes, sc, x, layout, k)
+            reps += 1
+            if time.perf_counter() - t0 > seconds or reps >= 50:
+                break
+        dt = time.perf_counter() - t0
+        if ctx is not None and hasattr(ctx, "unregister"):
+            ctx.unregister()
+        return nbytes * reps / dt / 1e9, reps, dt
+
+    ncpu, model = host_cpu()
+    v1, r1, d1 = leg(1)
+    va, ra, da = leg(ncpu)
+    return {"value": round(va, 4), "unit": "GB/s", "cores": ncpu, "kind": "oracle",
+            "sample": f"first {rows} rows of each of the {len(mats)} GEMVs of the step x {ra} passes ({da:.1f} s, "
+                      f"numpy fp64, {ncpu} threads)",
+            "one_thread": {"value": round(v1, 4), "unit": "GB/s", "cores": 1,
+                           "sample": f"the same sample x {r1} passes ({d1:.1f} s)"},
+            "host": {"nproc": ncpu, "cpu_model": model}}
+
+
+def record_traffic(csv_path):
+    """Writes profiles/traffic.json from an ncu --csv capture (one or more launches of the dominant
+    GEMV): dram read + write bytes per launch, keyed by the digest of the kernel source it ran."""
+    import csv
+    rows = list(csv.reader(open(csv_path)))
+    head = None
+    vals = {}
+    for r in rows:
+        if "Metric Name" in r and "Metric Value" in r:
+            head = r
+            continue
+        if head is None or len(r) != len(head):
+            continue
+        d = dict(zip(head, r))
+        if d.get("Metric Name") in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            unit = d.get("Metric Unit", "byte").lower()
+            scale = {"byte": 1, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9}.get(unit, 1)
+            v = float(d["Metric Value"].replace(",", "")) * scale
+            vals.setdefault(d.get("ID", "0"), {})[d["Metric Name"]] = v
+    per = [v.get("dram__bytes_read.sum", 0) + v.get("dram__bytes_write.sum", 0) for v in vals.values()]
+    if not per:
+        raise SystemExit("no dram__bytes metrics in " + csv_path)
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(path))
+    except Exception:
+        d = {}
+    key = os.environ.get("TRAFFIC_KEY", "gemv_t3_151936x4096_b1")
+    d[key] = {"dram_bytes_per_launch": int(round(statistics.median(per))), "launches": len(per),
+              "source": "tern_gemv_i8.cu", "source_sha": source_digest("tern_gemv_i8.cu"),
+              "note": "recorded by bench.py --record-traffic from an ncu capture of this source"}
+    with open(path, "w") as f:
+        json.dump(d, f, indent=1)
+    print(json.dumps({key: d[key]}))
 
 
 # -------------------------------------------------------------------------- the reference arm
@@ -622,14 +715,15 @@ def run_reference(args, rank, world):
         lim = None
     rows = 256
     samples, nbytes = [], 0
-    for li, layout in enumerate((O.Q2_0_G128, O.T3_5PB_G128)):
-        for mi, (n, k) in enumerate(LAYER_SET):
-            seed = synth.seed_for(2, mi) + 10 * layout
-            t = synth.ternary_codes(rows, k, seed)
-            s = synth.group_scales(rows, k // GROUP, seed)
-            x = synth.activations(1, k, seed)
-            samples.append((O.pack(t, layout), s, x, layout, k))
-            nbytes += rows * O.row_bytes(layout, k) + rows * (k // GROUP) * 2 + 2 * k + 2 * rows
+    cases = [(layout, mi, n, k) for layout in (O.Q2_0_G128, O.T3_5PB_G128) for mi, (n, k) in enumerate(LAYER_SET)]
+    cases.append((O.T3_5PB_G128, 3, LM_HEAD[0], LM_HEAD[1]))
+    for layout, mi, n, k in cases:
+        seed = synth.seed_for(2, mi) + 10 * layout
+        t = synth.ternary_codes(rows, k, seed)
+        s = synth.group_scales(rows, k // GROUP, seed)
+        x = synth.activations(1, k, seed)
+        samples.append((O.pack(t, layout), s, x, layout, k))
+        nbytes += rows * O.row_bytes(layout, k) + rows * (k // GROUP) * 2 + 2 * k + 2 * rows
 
     def step():
         for (codes, s, x, layout, k) in samples:
@@ -652,18 +746,29 @@ def run_reference(args, rank, world):
             "data": "synthetic (seeded, same distributions)",
             "config": {"workload": WORKLOAD, "batch": 1, "sample_rows_per_matrix": rows},
             "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{rows} rows of each of the six GEMVs per step (numpy fp64, 1 thread)"},
+                             "sample": f"{rows} rows of each of the seven GEMVs per step (numpy fp64, 1 thread)"},
             "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
+PROFILE_ALL = ["gemv_t3_151936x4096_b1", "gemv_q2_24576x4096_b1", "gemv_q2_34816x5120_b16", "gemm_q2_2048x17408x5120",
+               "gemm_t3_2048x17408x5120", "pack_q2_24576x4096", "pack_t3_24576x4096", "pack_q1_24576x4096",
+               "unpack_q2_24576x4096", "gemvt_q2_24576x4096_b1", "rotate_b64_k17408"]
+
+
 def run_profile_case(case: str, launches: int = 6):
-    """A handful of launches of one kernel, for an ncu capture (no timing claims)."""
+    """A handful of launches of one kernel case, for an ncu capture (no timing claims). 'all' runs
+    two launches of every case in PROFILE_ALL, one kernel family after another."""
     import torch
     import gemm_tern_gemv_b200 as T
+    if case == "all":
+        for c in PROFILE_ALL:
+            run_profile_case(c, 2)
+        return
     dev = torch.device("cuda", 0)
     parts = case.split("_")
-    kind, layout = parts[0], {"q2": T.Q2_0_G128, "t3": T.T3_5PB_G128, "q1": T.Q1_0_G128}[parts[1]]
+    kind = parts[0]
+    layout = {"q2": T.Q2_0_G128, "t3": T.T3_5PB_G128, "q1": T.Q1_0_G128}.get(parts[1])
     if kind == "gemv":
         n, k = (int(v) for v in parts[2].split("x"))
         b = int(parts[3][1:])
@@ -671,6 +776,12 @@ def run_profile_case(case: str, launches: int = 6):
         x = torch.randn((b, k), device=dev).to(torch.float16)
         ws = T.gemv_workspace(W, b)
         fn = lambda: T.gemv(W, x, workspace=ws, static_weights=True)
+    elif kind == "gemvt":
+        n, k = (int(v) for v in parts[2].split("x"))
+        b = int(parts[3][1:])
+        W = make_weights(torch, T, n, k, layout, 1, dev)
+        dy = torch.randn((b, n), device=dev).to(torch.float16)
+        fn = lambda: T.gemv_t(W, dy)
     elif kind == "gemm":
         m, n, k = (int(v) for v in parts[2].split("x"))
         W = make_weights(torch, T, n, k, layout, 1, dev)
@@ -682,6 +793,15 @@ def run_profile_case(case: str, launches: int = 6):
         s = (torch.randn((n, k // GROUP), device=dev).abs() * 0.02).to(torch.float16)
         Wp = T.pack(w, s, layout)
         fn = lambda: T.pack(w, s, layout, out=Wp)
+    elif kind == "unpack":
+        n, k = (int(v) for v in parts[2].split("x"))
+        W = make_weights(torch, T, n, k, layout, 1, dev)
+        fn = lambda: T.unpack(W, want_w=True, want_t=False)
+    elif kind == "rotate":
+        b, k = int(parts[1][1:]), int(parts[2][1:])
+        signs = torch.where(torch.rand(1024, device=dev) < 0.5, -1, 1).to(torch.int8)
+        xr = torch.randn((b, k), device=dev).to(torch.float16)
+        fn = lambda: T.hadamard_rotate(xr, signs)
     else:
         raise SystemExit(f"unknown case {case}")
     for _ in range(launches):
@@ -692,6 +812,9 @@ def run_profile_case(case: str, launches: int = 6):
 
 def main():
     args = parse()
+    if args.record_traffic:
+        record_traffic(args.record_traffic)
+        return
     if args.profile:
         run_profile_case(args.profile)
         return

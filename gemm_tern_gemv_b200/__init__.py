@@ -75,6 +75,7 @@ SIGNATURES = {
                                    ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "tern_hadamard_rotate": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
                                             ctypes.c_void_p, ctypes.c_void_p]),
+    "tern_device_result": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_int64]),
     "tern_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "tern_version": (ctypes.c_int32, []),
 }
@@ -105,6 +106,14 @@ def _status_string(status: int) -> str:
 def _check(status: int, what: str) -> None:
     if status != 0:
         raise TernError(status, what)
+
+
+def check_device_result(status=None, invalid_count=None) -> None:
+    """Reads back a device status word and / or an invalid-code counter and raises TernError with
+    TERN_ERR_TIMEOUT / TERN_ERR_INVALID_CODE when they report a failure (tern_device_result)."""
+    st = int(status.item()) & 0xFFFFFFFF if status is not None else 0
+    bad = int(invalid_count.item()) if invalid_count is not None else 0
+    _check(lib().tern_device_result(st, bad), "device result")
 
 
 def row_bytes(layout: int, k: int) -> int:

@@ -216,6 +216,12 @@ tern_status tern_hadamard_rotate(const uint16_t* x, int64_t batch, int64_t k, co
   return from_cuda(launch_rotate(x, batch, k, signs, y, static_cast<cudaStream_t>(stream)));
 }
 
+tern_status tern_device_result(uint32_t device_status, int64_t invalid_count) {
+  if (device_status & TERN_DEVICE_TIMEOUT) return TERN_ERR_TIMEOUT;
+  if (invalid_count > 0) return TERN_ERR_INVALID_CODE;
+  return TERN_OK;
+}
+
 const char* tern_status_string(tern_status status) {
   switch (status) {
     case TERN_OK: return "ok";

@@ -34,9 +34,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
-#include <map>
 #include <mutex>
-#include <tuple>
 
 #include "sm100.cuh"
 #include "tern_internal.cuh"
@@ -46,8 +44,11 @@ namespace {
 
 using sm100::smem_u32;
 
-constexpr int kI8MaxNW = 17;                  // consumer warps per CTA (one producer warp more)
-constexpr int kI8Threads = (kI8MaxNW + 1) * 32;
+// CTA shapes: one CTA of up to 17 consumer warps per SM, or two CTAs of up to 8 (each with its own
+// producer warp, ring and activation fragments). Two per SM overlap one CTA's prologue and drain with
+// the other's streaming, which pays on matrices with many tiles per SM; one per SM has the deeper ring.
+constexpr int kI8MaxNW1 = 17, kI8MaxNW2 = 8;
+__host__ __device__ constexpr int i8_max_nw(int cps) { return cps == 2 ? kI8MaxNW2 : kI8MaxNW1; }
 constexpr uint64_t kI8DefaultWaitNs = 1000000000ull;
 constexpr uint64_t kI8DrainNs = 200000000ull;  // bound on waiting for copies in flight at exit
 constexpr int kXV = 4;  // vectors of 8 activations a thread converts per row of x (slice <= 32 x threads)
@@ -220,8 +221,8 @@ __device__ __forceinline__ int a_k(int u, int m, int half, int q, int i) {
 // ---- the kernel ---------------------------------------------------------------------------------------
 // NPR: 1 = every consumer warp owns exactly one unit of each tile slice (activation fragments kept in
 // registers); 0 = any split (fragments read from shared memory per unit).
-template <int LAYOUT, int BATCH, int NPR>
-__global__ void __launch_bounds__(kI8Threads, 1)
+template <int LAYOUT, int BATCH, int NPR, int CPS>
+__global__ void __launch_bounds__((i8_max_nw(CPS) + 1) * 32, CPS)
     gemv_i8_kernel(const __grid_constant__ CUtensorMap mcf, const __grid_constant__ CUtensorMap mcr,
                    const __grid_constant__ CUtensorMap msc, const I8Params p) {
   using T = I8L<LAYOUT>;
@@ -382,7 +383,8 @@ __global__ void __launch_bounds__(kI8Threads, 1)
           D[2][i] = digits(v.z);
           D[3][i] = digits(v.w);
         }
-#pragma unroll
+        // this code runs once per launch, fetched cold: the plane loop stays rolled to keep it short
+#pragma unroll 1
         for (int pl = 0; pl < 4; pl++) {
           const uint32_t sel = (uint32_t)pl | ((uint32_t)(pl + 4) << 4);
           uint32_t w[4];
@@ -434,7 +436,7 @@ __global__ void __launch_bounds__(kI8Threads, 1)
           D[5][1][i] = 0;
         }
         // entry (unit, pair mp, lane (g = 4 sl + pl, qq)) word r = IMMA m = 2 mp + (r >> 1), half r & 1
-#pragma unroll
+#pragma unroll 1
         for (int pl = 0; pl < 4; pl++) {
           const uint32_t sel = (uint32_t)pl | ((uint32_t)(pl + 4) << 4);
 #pragma unroll
@@ -738,45 +740,15 @@ size_t i8_smem_bytes(const I8Params& p, int batch) {
   return s;
 }
 
-template <int LAYOUT, int BATCH, int NPR>
+template <int LAYOUT, int BATCH, int NPR, int CPS>
 const void* i8_kernel() {
-  return reinterpret_cast<const void*>(&gemv_i8_kernel<LAYOUT, BATCH, NPR>);
-}
-
-// Max clusters of `ks` CTAs with `smem` bytes each that can be resident at once (cached).
-int max_clusters(const void* kern, int ks, size_t smem) {
-  static std::mutex mu;
-  static std::map<std::tuple<const void*, int, size_t, int>, int> cache;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  const auto key = std::make_tuple(kern, ks, smem, dev);
-  std::lock_guard<std::mutex> lock(mu);
-  auto it = cache.find(key);
-  if (it != cache.end()) return it->second;
-  int n = 0;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) == cudaSuccess) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(ks * 148);
-    cfg.blockDim = dim3(kI8Threads);
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = ks;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
-  }
-  cudaGetLastError();
-  cache[key] = n;
-  return n;
+  return reinterpret_cast<const void*>(&gemv_i8_kernel<LAYOUT, BATCH, NPR, CPS>);
 }
 
 }  // namespace
 
-// Plan of the int8 kernel for (layout, n, k, batch) on `sms` SMs; ok = false when it does not apply.
-I8Plan i8_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
+// Plan for `cps` CTAs per SM; ok = false when nothing fits.
+static I8Plan i8_plan_cps(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms, int cps) {
   if (batch < 1 || batch > 2) return I8Plan{};
   const int unit_k = layout == TERN_T3_5PB_G128 ? 160 : 256;
   const int unit_b = layout == TERN_Q2_0_G128 ? 64 : 32;
@@ -787,7 +759,7 @@ I8Plan i8_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
   const int units = (int)(rb / unit_b);
   const int tiles = (int)((n + 15) / 16);
   const int groups = (int)(k / kGroup);
-  const size_t cap = 227 * 1024;
+  const size_t cap = (size_t)(228 / cps - 1) * 1024;
   I8Plan best{};
   double best_cost = 1e300;
   // cost of a K split ks: tiles per cluster x units per warp, fewer than 16 warps counted as slower
@@ -817,9 +789,9 @@ I8Plan i8_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
     pl.code_bytes = 16 * slice_b;
     pl.stage_bytes = (pl.code_bytes + 16 * pl.sc_w * 2 + 1023) / 1024 * 1024;
     pl.xk = (L * unit_k + 7) / 8 * 8;
-    const int clusters = std::max(1, sms / ks);
+    const int clusters = std::max(1, cps * sms / ks);
     pl.tmax = (tiles + clusters - 1) / clusters;
-    for (int nw = std::min(L, 8); nw <= std::min(L, kI8MaxNW); nw++) {
+    for (int nw = std::min(L, 8); nw <= std::min(L, i8_max_nw(cps)); nw++) {
       if (pl.xk > kXV * 8 * (nw + 1) * 32) continue;  // every activation of the slice converted in one pass
       const size_t fixed = 1024 + 48 + 4 * (size_t)batch * pl.xk + (size_t)L * ent_bytes * batch + 128 * (size_t)batch +
                            (layout == TERN_Q1_0_G128 ? 8 * (size_t)L * batch : 0) + 64 * (size_t)pl.tmax * nw * batch;
@@ -827,8 +799,8 @@ I8Plan i8_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
       // the slowest warp sets the tile time; an SM streams faster the more warps it has (measured: 16
       // warps with one or two units each beat 13 warps with two each), so fewer warps count as slower
       const int per_warp = (L + nw - 1) / nw;
-      const double cost = (double)pl.tmax * per_warp * (16.0 / std::min(16, nw)) * (1.0 + 0.02 * (ks - 1)) +
-                          0.001 * std::abs(nw - 16);
+      const double cost = (double)pl.tmax * per_warp * (16.0 / std::min(16, cps * nw)) * (1.0 + 0.02 * (ks - 1)) +
+                          0.001 * std::abs(cps * nw - 16);
       if (cost < best_cost) {
         best_cost = cost;
         best = pl;
@@ -836,15 +808,26 @@ I8Plan i8_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
         best.npr = (L % nw == 0 && L / nw == 1) ? 1 : 0;
         best.stages = (int)std::min<size_t>(8, (cap - fixed) / (pl.stage_bytes + 16));
         best.ok = true;
+        best.cps = cps;
       }
     }
   }
   return best;
 }
 
+// Plan of the int8 kernel for (layout, n, k, batch) on `sms` SMs; ok = false when it does not apply.
+// Two CTAs per SM when one per SM would give each SM at least 14 row tiles or split K over a cluster
+// (measured: the LM head and the 27B-class matrices gain 10-20 %, the 8B-class ones lose).
+I8Plan i8_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
+  const I8Plan one = i8_plan_cps(layout, n, k, batch, sms, 1);
+  if (one.ok && one.tmax < 14 && one.ks == 1) return one;
+  const I8Plan two = i8_plan_cps(layout, n, k, batch, sms, 2);
+  return two.ok ? two : one;
+}
+
 namespace {
 
-template <int LAYOUT, int BATCH, int NPR>
+template <int LAYOUT, int BATCH, int NPR, int CPS>
 cudaError_t launch_i8_t(const tern_matrix& W, const uint16_t* x, uint16_t* y, const I8Plan& pl, cudaStream_t st,
                         uint32_t flags, uint32_t* status, uint64_t wait_ns) {
   using T = I8L<LAYOUT>;
@@ -872,17 +855,12 @@ cudaError_t launch_i8_t(const tern_matrix& W, const uint16_t* x, uint16_t* y, co
   p.tmax = pl.tmax;
   p.xk = pl.xk;
   const size_t smem = i8_smem_bytes<LAYOUT>(p, BATCH);
-  const void* kern = i8_kernel<LAYOUT, BATCH, NPR>();
-  // clusters resident at once (a K split needs its CTAs co-scheduled); never more than one wave
-  int clusters = std::max(1, sm_count() / pl.ks);
-  const int mc = max_clusters(kern, pl.ks, smem);
-  if (mc > 0) clusters = std::min(clusters, mc);
-  if ((pl.tiles + clusters - 1) / clusters > pl.tmax) {
-    // fewer clusters than planned: every cluster owns more tiles than the partial-sum space holds
-    p.tmax = (pl.tiles + clusters - 1) / clusters;
-  }
-  const size_t smem2 = i8_smem_bytes<LAYOUT>(p, BATCH);
-  if (smem2 > 227 * 1024 + 1024) return cudaErrorInvalidValue;
+  const void* kern = i8_kernel<LAYOUT, BATCH, NPR, CPS>();
+  // the planned grid: clusters own disjoint tiles and never wait on one another, so clusters that
+  // do not fit at once simply run in a later wave
+  const int clusters = std::max(1, CPS * sm_count() / pl.ks);
+  if ((pl.tiles + clusters - 1) / clusters > pl.tmax) return cudaErrorInvalidValue;  // plan and device disagree
+  const size_t smem2 = smem;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2);
   if (e != cudaSuccess) return e;
   // tensor maps: codes as 32-bit words [n][row bytes / 4] (boxes box_b / 4 and rem_b / 4 wide, 16 rows);
@@ -919,18 +897,24 @@ cudaError_t launch_i8_t(const tern_matrix& W, const uint16_t* x, uint16_t* y, co
   cfg.attrs = at;
   cfg.numAttrs = na;
   (void)T::kUnitK;
-  e = cudaLaunchKernelEx(&cfg, gemv_i8_kernel<LAYOUT, BATCH, NPR>, mcf, mcr, msc, p);
+  e = cudaLaunchKernelEx(&cfg, gemv_i8_kernel<LAYOUT, BATCH, NPR, CPS>, mcf, mcr, msc, p);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
+template <int LAYOUT, int CPS>
+cudaError_t launch_i8_c(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y, const I8Plan& pl,
+                        cudaStream_t st, uint32_t flags, uint32_t* status, uint64_t wait_ns) {
+  if (batch == 1)
+    return pl.npr ? launch_i8_t<LAYOUT, 1, 1, CPS>(W, x, y, pl, st, flags, status, wait_ns)
+                  : launch_i8_t<LAYOUT, 1, 0, CPS>(W, x, y, pl, st, flags, status, wait_ns);
+  return pl.npr ? launch_i8_t<LAYOUT, 2, 1, CPS>(W, x, y, pl, st, flags, status, wait_ns)
+                : launch_i8_t<LAYOUT, 2, 0, CPS>(W, x, y, pl, st, flags, status, wait_ns);
+}
 template <int LAYOUT>
 cudaError_t launch_i8_l(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y, const I8Plan& pl,
                         cudaStream_t st, uint32_t flags, uint32_t* status, uint64_t wait_ns) {
-  if (batch == 1)
-    return pl.npr ? launch_i8_t<LAYOUT, 1, 1>(W, x, y, pl, st, flags, status, wait_ns)
-                  : launch_i8_t<LAYOUT, 1, 0>(W, x, y, pl, st, flags, status, wait_ns);
-  return pl.npr ? launch_i8_t<LAYOUT, 2, 1>(W, x, y, pl, st, flags, status, wait_ns)
-                : launch_i8_t<LAYOUT, 2, 0>(W, x, y, pl, st, flags, status, wait_ns);
+  return pl.cps == 2 ? launch_i8_c<LAYOUT, 2>(W, x, batch, y, pl, st, flags, status, wait_ns)
+                     : launch_i8_c<LAYOUT, 1>(W, x, batch, y, pl, st, flags, status, wait_ns);
 }
 
 }  // namespace

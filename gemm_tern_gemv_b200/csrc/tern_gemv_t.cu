@@ -151,12 +151,30 @@ __global__ void __launch_bounds__(kTThreads) gemv_t_kernel(const uint8_t* __rest
   }
 }
 
+// Sums the slices' fp32 partials of 32 consecutive outputs per CTA: the 8 warps take every eighth
+// slice (loads of one warp are 128 contiguous bytes, four in flight per lane), then one warp adds the
+// 8 warp sums. The order is fixed (slices sg, sg + 8, ... within warp sg, then warps 0..7), so the
+// result depends only on the inputs.
 __global__ void __launch_bounds__(256) gemv_t_reduce(const float* __restrict__ part, int slices, int64_t total,
                                                      uint16_t* dx) {
-  for (int64_t e = blockIdx.x * 256 + threadIdx.x; e < total; e += (int64_t)gridDim.x * 256) {
+  __shared__ float red[8][33];
+  const int c = threadIdx.x & 31, sg = threadIdx.x >> 5;
+  for (int64_t e0 = (int64_t)blockIdx.x * 32; e0 < total; e0 += (int64_t)gridDim.x * 32) {
+    const int64_t e = e0 + c;
     float v = 0.f;
-    for (int s = 0; s < slices; s++) v += part[(int64_t)s * total + e];
-    dx[e] = __half_as_ushort(__float2half_rn(v));
+    if (e < total) {
+#pragma unroll 4
+      for (int s = sg; s < slices; s += 8) v += part[(int64_t)s * total + e];
+    }
+    red[sg][c] = v;
+    __syncthreads();
+    if (sg == 0 && e < total) {
+      float t = red[0][c];
+#pragma unroll
+      for (int j = 1; j < 8; j++) t += red[j][c];
+      dx[e] = __half_as_ushort(__float2half_rn(t));
+    }
+    __syncthreads();
   }
 }
 
@@ -176,8 +194,8 @@ cudaError_t launch_t(const tern_matrix& W, const uint16_t* dy, int batch, uint16
   e = cudaGetLastError();
   if (e != cudaSuccess || p.slices == 1) return e;
   const int64_t total = (int64_t)batch * W.k;
-  const int64_t blocks = (total + 255) / 256;
-  gemv_t_reduce<<<(unsigned)(blocks < 4 * sm_count() ? blocks : 4 * sm_count()), 256, 0, st>>>(part, p.slices,
+  const int64_t blocks = (total + 31) / 32;
+  gemv_t_reduce<<<(unsigned)(blocks < 8 * sm_count() ? blocks : 8 * sm_count()), 256, 0, st>>>(part, p.slices,
                                                                                               total, dx);
   return cudaGetLastError();
 }

@@ -46,6 +46,7 @@ struct I8Plan {
   int code_bytes, stage_bytes, stages;
   int xk;          // activations per CTA (halves)
   int tmax;        // tiles per cluster (upper bound)
+  int cps;         // CTAs per SM (1 or 2)
 };
 I8Plan i8_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms);
 // status / wait_ns: optional device status word and bound on each pipeline wait (0 = 1 s)

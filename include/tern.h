@@ -68,8 +68,8 @@ typedef enum tern_status {
   TERN_ERR_UNSUPPORTED = 2,   /* unknown layout id, or a layout/size this entry point lacks */
   TERN_ERR_ALIGNMENT = 3,     /* pointer or stride not 16-byte aligned */
   TERN_ERR_WORKSPACE = 4,     /* split-K workspace missing or smaller than required */
-  TERN_ERR_INVALID_CODE = 5,  /* reserved for callers that turn an invalid-code count into a status */
-  TERN_ERR_TIMEOUT = 6,       /* reserved for callers that turn a device timeout flag into a status */
+  TERN_ERR_INVALID_CODE = 5,  /* tern_device_result: tern_unpack counted invalid codes */
+  TERN_ERR_TIMEOUT = 6,       /* tern_device_result: a pipeline wait of a product ran out */
   TERN_ERR_CUDA = 7           /* a CUDA runtime call or kernel launch failed */
 } tern_status;
 
@@ -79,7 +79,7 @@ typedef enum tern_layout {
   TERN_Q1_0_G128 = 3
 } tern_layout;
 
-/* Bits of the device status word that tern_gemm writes (atomic OR) when it is non-NULL. */
+/* Bits of the device status word that tern_gemm and tern_gemv_opt write (atomic OR) when given one. */
 #define TERN_DEVICE_TIMEOUT 1u   /* a pipeline wait exceeded its bound; the tile was abandoned */
 
 /* A packed ternary matrix W[n][k] (n output features, k reduction length). Host struct holding
@@ -97,11 +97,15 @@ typedef struct tern_matrix {
 /* ---- size arithmetic (host only, no CUDA) ------------------------------------------------ */
 
 /* Minimum packed row stride in bytes: K/4 for Q2_0_g128, ceil(K/5) rounded up to 16 for base-3,
- * K/8 for Q1_0_g128.
+ * K/8 for Q1_0_g128 (the containers of "Ternary Bonsai 2 27B ..." discuss.pytorch.kr, section "두
+ * 가지 패킹: PTQ1_0과 PQ2_0": 2-bit slots, dense trits; "Bonsai 27B와 1비트가 살아남는 법" velog.io,
+ * section "ternary와 binary가 뭔가": one bit per binary weight; codes only, scales are separate).
  * Returns -1 for an unknown layout or K not a positive multiple of 128. */
 TERN_API int64_t tern_row_bytes(int32_t layout, int64_t k);
 
-/* n * tern_row_bytes(layout, k): bytes of packed codes at the minimum stride (scales excluded).
+/* n * tern_row_bytes(layout, k): bytes of packed codes at the minimum stride (scales excluded); with
+ * n * (k/128) * 2 bytes of scales this is what a product streams per call (section "두 가지 패킹" of
+ * the page above gives the per-128-weight container sizes it is checked against).
  * Returns -1 on invalid arguments. */
 TERN_API int64_t tern_packed_bytes(int32_t layout, int64_t n, int64_t k);
 
@@ -148,7 +152,10 @@ TERN_API tern_status tern_pack_flips(int32_t layout, int64_t n, int64_t k, const
 
 /* ---- unpack (test / debug path; the products never call it) ------------------------------ */
 
-/* Expands W to dense form. Either output may be NULL, not both.
+/* Expands W to dense form: w = s * t per weight ("Bonsai 27B와 1비트가 살아남는 법", section "포맷의
+ * 정체", eq. w_i = s_g * t_i), the exact inverse of tern_pack on its codes ("Metal 환경에서 ... Bonsai
+ * 8B를 파인튜닝", paragraph "그것을 파인튜닝하는 방법": lossless re-encode). Either output may be NULL,
+ * not both.
  *   w_out          device fp16 [n][w_row_stride]: s * t (exact in fp16), 0 for invalid codes
  *   t_out          device int8 [n][t_row_stride]: t, 0 for invalid codes (t_row_stride bytes)
  *   invalid_count  device int32 or NULL: the number of weights with an invalid code is ADDED to
@@ -159,16 +166,22 @@ TERN_API tern_status tern_unpack(const tern_matrix* W, uint16_t* w_out, int64_t 
 
 /* ---- decode GEMV (batch 1..64) -------------------------------------------------------------- */
 
-/* Bytes of split-K workspace tern_gemv needs for this matrix and batch (0 when it needs none).
+/* Bytes of split-K workspace tern_gemv needs for this matrix and batch (0 when it needs none; batches
+ * 1-2 of matrices whose rows are whole 32- or 64-byte units split K over thread-block clusters
+ * instead). The product is the decode GEMV of "Ternary Bonsai 2 27B ..." discuss.pytorch.kr, section
+ * "처리량" (batch-1 token generation).
  * Depends only on (W->layout, W->n, W->k, batch) and the current device's SM count.
  * Returns 0 also for invalid arguments (tern_gemv then reports the error). */
 TERN_API size_t tern_gemv_workspace_bytes(const tern_matrix* W, int64_t batch);
 
-/* y[b][n] = sum_g s[n][g] * sum_{k in group g} t[n][k] * x[b][k] for b < batch; fp32
- * accumulation, fp16 result. Small batches run on mma.sync kernels that decode the codes in
- * registers; batches of 17 or more with n % 8 == 0 run on the tcgen05 kernel of tern_gemm (no
- * workspace); so do Q1_0_g128 batches of 5 or more with n % 8 == 0. Other Q1_0_g128 batches run
- * as one register-kernel launch per two rows of x.
+/* y[b][n] = sum_g s[n][g] * sum_{k in group g} t[n][k] * x[b][k] for b < batch ("Ternary Bonsai 2
+ * 27B ..." discuss.pytorch.kr, section "그룹 단위 스케일을 공유하는 삼진 형식", eq. w_i = s_g t_i; the
+ * packed codes are read directly and unpack and group scale are fused, section "하이브리드 어텐션을
+ * 위한 저비트 커널"); the activations' own precision is kept (x exact as int8 planes or fp16), fp32
+ * accumulation, fp16 result. Batches 1-2 run on int8 mma.sync kernels fed by TMA (K split over a
+ * cluster for narrow matrices); batches 3-16 on fp16 mma.sync kernels; batches of 17 or more with
+ * n % 8 == 0 on the tcgen05 kernel of tern_gemm (no workspace), as do Q1_0_g128 batches of 5 or
+ * more with n % 8 == 0. Other Q1_0_g128 batches run as one launch per two rows of x.
  * The result of a call depends only on (W, x, batch) and the device.
  *   x          device fp16 [batch][k], contiguous
  *   y          device fp16 [batch][n], contiguous
@@ -243,9 +256,10 @@ TERN_API tern_status tern_gemv_noalloc(const tern_matrix* W, const uint16_t* x, 
 
 /* ---- prefill GEMM on tcgen05 tensor cores --------------------------------------------------- */
 
-/* Y[m][n] = sum_k X[m][k] * s[n][k/128] * t[n][k]; packed tiles are decoded to fp16 s*t (exact)
- * in shared memory and multiplied on the 5th-generation tensor cores with fp32 accumulation in
- * tensor memory.
+/* Y[m][n] = sum_k X[m][k] * s[n][k/128] * t[n][k], the prefill (prompt-processing) product of
+ * "Ternary Bonsai 2 27B ..." discuss.pytorch.kr, section "처리량" (pp512, compute-bound); packed tiles
+ * are decoded to fp16 s*t (exact) in shared memory and multiplied on the 5th-generation tensor
+ * cores with fp32 accumulation in tensor memory.
  *   X              device fp16 [m][k], contiguous;  Y device fp16 [m][n], contiguous
  *   device_status  device uint32 or NULL: TERN_DEVICE_TIMEOUT is OR-ed in if an internal pipeline
  *                  wait exceeds its bound (the kernel then abandons its work and exits; Y is
@@ -295,6 +309,15 @@ TERN_API tern_status tern_gemv_t(const tern_matrix* W, const uint16_t* dy, int64
  *         batch * k too large), TERN_ERR_ALIGNMENT (x or y not 2-byte aligned), TERN_ERR_CUDA. */
 TERN_API tern_status tern_hadamard_rotate(const uint16_t* x, int64_t batch, int64_t k, const int8_t* signs,
                                           uint16_t* y, void* stream);
+
+/* Turns the device-side results a caller has read back into a status, so that a failure is refused
+ * loudly ("Ternary Bonsai 2 27B ..." discuss.pytorch.kr, the runtime notes after section "블록 단위
+ * 하다마드 회전": a runtime must reject what it cannot carry out, not emit garbage):
+ *   device_status  the value of the status word given to tern_gemm / tern_gemv_opt
+ *   invalid_count  the value of the counter given to tern_unpack (0 if none)
+ * Returns TERN_ERR_TIMEOUT if TERN_DEVICE_TIMEOUT is set, else TERN_ERR_INVALID_CODE if
+ * invalid_count > 0, else TERN_OK. Host only; makes no CUDA call. */
+TERN_API tern_status tern_device_result(uint32_t device_status, int64_t invalid_count);
 
 /* Static description of a status code (never NULL). */
 TERN_API const char* tern_status_string(tern_status status);

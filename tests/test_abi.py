@@ -239,3 +239,23 @@ def test_noalloc_scratch_claim_of_the_header(lib):
                 for n in (1000, 5120, 34816, 151936 if k == 4096 else 34816):
                     m = _mat(layout=layout, n=n, k=k, code_row_stride=rb(k), scale_row_stride=k // 128)
                     assert lib.tern_gemv_workspace_bytes(ctypes.byref(m), b) <= limit
+
+
+def test_device_result_turns_device_words_into_statuses(lib):
+    # TERN_DEVICE_TIMEOUT wins over an invalid-code count; both map to the reserved statuses
+    assert lib.tern_device_result(0, 0) == 0
+    assert lib.tern_device_result(1, 0) == 6   # TERN_ERR_TIMEOUT
+    assert lib.tern_device_result(1, 5) == 6
+    assert lib.tern_device_result(0, 3) == 5   # TERN_ERR_INVALID_CODE
+    assert lib.tern_device_result(2, 0) == 0   # bits other than TERN_DEVICE_TIMEOUT are not errors
+    assert lib.tern_device_result(0, -1) == 0
+
+
+def test_gemv_opt_rejects_before_launch(lib):
+    import gemm_tern_gemv_b200 as T
+    m = _mat()
+    args = (ctypes.byref(m), ctypes.c_void_p(FAKE), 1, ctypes.c_void_p(FAKE), None, 0)
+    bad_flag = T.TernGemvOptsC(2, None, 0)
+    assert lib.tern_gemv_opt(*args, ctypes.byref(bad_flag), None) == 1
+    misaligned = T.TernGemvOptsC(0, FAKE + 2, 0)
+    assert lib.tern_gemv_opt(*args, ctypes.byref(misaligned), None) == 3

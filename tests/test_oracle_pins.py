@@ -94,6 +94,25 @@ def test_q2_byte_table_exhaustive():
     assert valid == 3**4
 
 
+def test_q2_count_invalid_is_the_number_of_0b10_fields():
+    # every byte value in the first byte of its row; the count must equal the number of 2-bit fields
+    # equal to 0b10 (the one invalid code), counted here bit by bit, independently of the oracle
+    codes = np.zeros((256, 32), dtype=np.uint8)
+    codes[:, 0] = np.arange(256)
+    expected = 0
+    for byte in range(256):
+        for i in range(4):
+            hi, lo = (byte >> (2 * i + 1)) & 1, (byte >> (2 * i)) & 1
+            expected += int(hi == 1 and lo == 0)
+    assert expected == 4 * 64  # each field position holds 0b10 in a quarter of the 256 bytes
+    assert O.count_invalid(codes, O.Q2_0_G128, 256, 128) == expected
+    # per row, including bytes past the first and rows with several invalid fields
+    for byte in (0x02, 0x08, 0x20, 0x80, 0xAA, 0x55, 0xFF, 0x00):
+        row = np.full((1, 32), byte, dtype=np.uint8)
+        per_byte = sum(((byte >> (2 * i)) & 3) == 2 for i in range(4))
+        assert O.count_invalid(row, O.Q2_0_G128, 1, 128) == 32 * per_byte
+
+
 def test_t3_byte_table_exhaustive():
     codes = np.full((256, 32), O.T3_PAD_BYTE, dtype=np.uint8)
     codes[:, 0] = np.arange(256)
