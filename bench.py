@@ -55,6 +55,10 @@ def parse():
     p.add_argument("--warmup", type=int, default=50)
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--no-extras", action="store_true", help="skip the per-row measurements of the other kernels")
+    p.add_argument("--eager", action="store_true",
+                   help="launch each step's GEMVs directly instead of replaying the step's CUDA graph (the same "
+                        "kernels and arguments; used for the ncu launch list, whose per-kernel replay of graph "
+                        "nodes does not launch the thread-block-cluster kernels)")
     p.add_argument("--profile", default=None, metavar="CASE",
                    help="run a few launches of one kernel case for ncu: gemv_{q2|t3|q1}_NxK_bB, "
                         "gemm_{q2|t3|q1}_MxNxK, pack_{q2|t3|q1}_NxK, unpack_{q2|t3|q1}_NxK, "
@@ -290,9 +294,15 @@ def run_native(args, rank, world, local_rank):
             torch.distributed.barrier()
         torch.cuda.synchronize()
 
+    def run_step(i):
+        if args.eager:
+            step(i % copies)
+        else:
+            graphs[i % copies].replay()
+
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
-            graphs[i % copies].replay()
+            run_step(i)
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -304,7 +314,7 @@ def run_native(args, rank, world, local_rank):
         with torch.cuda.stream(stream):
             e0.record(stream)
             for i in range(args.steps):
-                graphs[i % copies].replay()
+                run_step(i)
             e1.record(stream)
             clk.sample_now()  # one sample while the queued replays run, however short the region
         e1.synchronize()
@@ -343,7 +353,8 @@ def run_native(args, rank, world, local_rank):
                                  f"{l2 / 1e6:.0f} MB)", "parallelism": f"replicas x{world}",
                            "hbm_frac_of_8TBps": round(value / world / 8000.0, 4),
                            "launch": "tern_gemv_ex with TERN_GEMV_STATIC_WEIGHTS (programmatic dependent launch: "
-                                     "each GEMV starts streaming its weights while the previous one finishes)"},
+                                     "each GEMV starts streaming its weights while the previous one finishes)",
+                           "step_launch": "eager launches" if args.eager else "one CUDA graph replay per step"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary()}
         if extras:

@@ -69,6 +69,7 @@ struct I8Params {
   int units;          // units per row
   int L;              // units per K slice (the last slice may be shorter)
   int nw;             // consumer warps
+  uint32_t nw_rcp;    // floor(2^20 / nw) + 1: x / nw = (x * nw_rcp) >> 20 for 0 <= x < 2^20 / nw
   int early;          // weight tiles may be requested before the preceding grid completes
   int box_b, nfull, rem_b;  // code boxes of one stage: nfull x box_b bytes, then rem_b bytes (0 = none)
   int sc_w;           // scale box width (halves, multiple of 8)
@@ -89,6 +90,19 @@ __device__ __forceinline__ void imma_u8(int (&d)[4], uint32_t a0, uint32_t a1, u
   asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
                : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// The same products with a zero accumulator (the first IMMA of a chain: no register has to be cleared).
+__device__ __forceinline__ void imma_s8_z(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                          uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};\n"
+               : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
+}
+__device__ __forceinline__ void imma_u8_z(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                          uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};\n"
+               : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
 }
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
   uint4 v;
@@ -484,8 +498,14 @@ __global__ void __launch_bounds__((i8_max_nw(CPS) + 1) * 32, CPS)
     }
   } else {
     // ---- consumers ------------------------------------------------------------------------------
+    // Chunk c of a stage is local units [c nu / NW, (c + 1) nu / NW). With NPR every warp keeps its
+    // own chunk (one unit); otherwise warp w takes chunk (w + i) mod NW in stage i, so a warp with a
+    // larger chunk in one stage has a smaller one in the next and no warp runs ahead of the others by
+    // more than one chunk (the chunks differ by one unit when NW does not divide nu).
     const int nu = u1 - u0;
-    const int ub = (int)((int64_t)warp * nu / NW), ue = (int)((int64_t)(warp + 1) * nu / NW);  // local units
+    int ck = warp;
+    auto chunk_lo = [&](int c) { return (int)(((uint32_t)(c * nu) * p.nw_rcp) >> 20); };
+    int ub = chunk_lo(ck), ue = chunk_lo(ck + 1);
     const bool bval = kEnt == 32 || ((g >> 2) == (q >> 1));
     const uint32_t fbase = smem_u32(frag) + (uint32_t)(kEnt == 32 ? lane : (q * 4 + (g & 3))) * 16u;
     uint32_t mul[4];
@@ -504,34 +524,45 @@ __global__ void __launch_bounds__((i8_max_nw(CPS) + 1) * 32, CPS)
     for (int b = 0; b < BATCH; b++)  // 2^-S (base-3) or 2^(-S-6) (the A values of Q2 / binary are 64 t / 128 b)
       outscale[b] = plane_w * __uint_as_float((uint32_t)(127 - S[b] - (LAYOUT == TERN_T3_5PB_G128 ? 0 : 6)) << 23);
     // Shared-memory addresses of a local unit within a stage; every tile has the same layout, so
-    // they are computed once per unit (once per warp when it owns a single unit), with shifts only:
-    // a slice is one box (box_b = slice bytes <= 1 KB) or 1 KB boxes plus a narrower last one.
+    // they depend on the unit and the lane only: a slice is one box (box_b = slice bytes <= 1 KB) or
+    // 1 KB boxes plus a narrower last one.
     const bool box1k = p.box_b == 1024;
     const uint32_t box_stride = 16u * (uint32_t)p.box_b;
     const uint32_t frag_unit = (uint32_t)(kMP * BATCH * kEnt) * 16u;
+    const int lane_off = q * (T::kUnitB / 4);
+    const uint32_t cR_one = (uint32_t)(g * p.box_b + lane_off);             // one-box slices
+    const uint32_t c8_one = 8u * (uint32_t)p.box_b;
+    const uint32_t sR_lane = (uint32_t)(p.code_bytes + (g * p.sc_w - sx0) * 2);
     struct UA {
       uint32_t cR, c8, sR, fr;  // codes of row g, row-8 distance, scale of row g, fragments
       bool sval;
     };
     auto unit_addr = [&](int ul) -> UA {
       UA a;
-      const int off = ul * T::kUnitB + q * (T::kUnitB / 4);
-      const int bo = box1k ? (off >> 10) : 0;
-      const uint32_t width = (uint32_t)(bo < p.nfull ? p.box_b : p.rem_b);
-      a.cR = (uint32_t)bo * box_stride + (uint32_t)g * width + (uint32_t)(off - (bo << 10) * (box1k ? 1 : 0));
-      a.c8 = 8u * width;
+      if (box1k) {
+        const int off = ul * T::kUnitB + lane_off;
+        const int bo = off >> 10;
+        const uint32_t width = (uint32_t)(bo < p.nfull ? p.box_b : p.rem_b);
+        a.cR = (uint32_t)bo * box_stride + (uint32_t)g * width + (uint32_t)(off & 1023);
+        a.c8 = 8u * width;
+      } else {
+        a.cR = cR_one + (uint32_t)(ul * T::kUnitB);
+        a.c8 = c8_one;
+      }
       const int u = u0 + ul;
       int grp;
       a.sval = true;
       if (LAYOUT == TERN_T3_5PB_G128) {
-        const int g0 = (160 * u) >> 7, gl = (160 * u + 159) >> 7;  // kGroup = 128
+        // a unit starts 0, 32, 64 or 96 trits into group (160 u) / 128 and always reaches the next
+        // group; slot 1 carries no data when that group is past K
+        const int g0 = (5 * u) >> 2;  // (160 u) / 128
         grp = g0 + (q >> 1);
-        a.sval = grp <= gl && grp < p.groups;  // slot 1 of a unit inside one group carries no data
+        a.sval = grp < p.groups;
         if (!a.sval) grp = g0;
       } else {
         grp = 2 * u + (q >> 1);
       }
-      a.sR = (uint32_t)(p.code_bytes + (g * p.sc_w + (grp - sx0)) * 2);
+      a.sR = sR_lane + (uint32_t)grp * 2u;
       a.fr = fbase + (uint32_t)ul * frag_unit;
       return a;
     };
@@ -563,6 +594,11 @@ __global__ void __launch_bounds__((i8_max_nw(CPS) + 1) * 32, CPS)
     uint32_t ph = 0;
     for (int i = 0; i < nt; i++) {
       const uint32_t st = ring + (uint32_t)s * (uint32_t)p.stage_bytes;
+      if (!NPR && i > 0) {
+        if (++ck == NW) ck = 0;
+        ub = ck ? ue : 0;
+        ue = chunk_lo(ck + 1);
+      }
       if (!mbar_wait(full0 + 8u * s, ph, abort_flag, p.status, p.wait_ns)) break;
       float acc[BATCH][2];
 #pragma unroll
@@ -595,6 +631,8 @@ __global__ void __launch_bounds__((i8_max_nw(CPS) + 1) * 32, CPS)
           for (int b = 0; b < BATCH; b++) {
             if (NPR) {
               bf[mp][b] = breg[mp][b];
+            } else if (kEnt == 32) {
+              bf[mp][b] = lds128(ua.fr + (uint32_t)((mp * BATCH + b) * kEnt) * 16u);
             } else {
               bf[mp][b] = make_uint4(0, 0, 0, 0);
               lds128_if(bf[mp][b], ua.fr + (uint32_t)((mp * BATCH + b) * kEnt) * 16u, bval);
@@ -602,8 +640,6 @@ __global__ void __launch_bounds__((i8_max_nw(CPS) + 1) * 32, CPS)
           }
         // two independent accumulator chains (even / odd IMMA) halve the dependent MMA latency
         int c[BATCH][4], cx[BATCH][4];
-#pragma unroll
-        for (int b = 0; b < BATCH; b++) c[b][0] = c[b][1] = c[b][2] = c[b][3] = cx[b][0] = cx[b][1] = cx[b][2] = cx[b][3] = 0;
         if constexpr (LAYOUT == TERN_Q2_0_G128) {
 #pragma unroll
           for (int m = 0; m < 8; m++) {
@@ -613,7 +649,9 @@ __global__ void __launch_bounds__((i8_max_nw(CPS) + 1) * 32, CPS)
 #pragma unroll
             for (int b = 0; b < BATCH; b++) {
               const uint4& bb = bf[m >> 1][b];
-              if (m & 1) imma_s8(cx[b], a0, a1, a2, a3, bb.z, bb.w);
+              if (m == 0) imma_s8_z(c[b], a0, a1, a2, a3, bb.x, bb.y);
+              else if (m == 1) imma_s8_z(cx[b], a0, a1, a2, a3, bb.z, bb.w);
+              else if (m & 1) imma_s8(cx[b], a0, a1, a2, a3, bb.z, bb.w);
               else imma_s8(c[b], a0, a1, a2, a3, bb.x, bb.y);
             }
           }
@@ -626,7 +664,9 @@ __global__ void __launch_bounds__((i8_max_nw(CPS) + 1) * 32, CPS)
 #pragma unroll
             for (int b = 0; b < BATCH; b++) {
               const uint4& bb = bf[m >> 1][b];
-              if (m & 1) imma_u8(cx[b], a0, a1, a2, a3, bb.z, bb.w);
+              if (m == 0) imma_u8_z(c[b], a0, a1, a2, a3, bb.x, bb.y);
+              else if (m == 1) imma_u8_z(cx[b], a0, a1, a2, a3, bb.z, bb.w);
+              else if (m & 1) imma_u8(cx[b], a0, a1, a2, a3, bb.z, bb.w);
               else imma_u8(c[b], a0, a1, a2, a3, bb.x, bb.y);
             }
           }
@@ -659,7 +699,9 @@ __global__ void __launch_bounds__((i8_max_nw(CPS) + 1) * 32, CPS)
 #pragma unroll
             for (int b = 0; b < BATCH; b++) {
               const uint4& bb = bf[m >> 1][b];
-              if (m & 1) imma_u8(cx[b], a0, a1, a2, a3, bb.z, bb.w);
+              if (m == 0) imma_u8_z(c[b], a0, a1, a2, a3, bb.x, bb.y);
+              else if (m == 1) imma_u8_z(cx[b], a0, a1, a2, a3, bb.z, bb.w);
+              else if (m & 1) imma_u8(cx[b], a0, a1, a2, a3, bb.z, bb.w);
               else imma_u8(c[b], a0, a1, a2, a3, bb.x, bb.y);
             }
           }
@@ -844,6 +886,10 @@ cudaError_t launch_i8_t(const tern_matrix& W, const uint16_t* x, uint16_t* y, co
   p.units = pl.units;
   p.L = pl.L;
   p.nw = pl.nw;
+  // chunk bounds c nu / nw by a reciprocal: exact while nw^2 L < 2^20 (then (c nu) e < 2^20 with
+  // e = nw_rcp nw - 2^20 <= nw), far above any slice a plan holds
+  p.nw_rcp = (1u << 20) / (uint32_t)pl.nw + 1u;
+  if ((int64_t)pl.nw * pl.nw * pl.L >= (1 << 20)) return cudaErrorInvalidValue;
   p.early = (flags & TERN_GEMV_STATIC_WEIGHTS) ? 1 : 0;
   p.box_b = pl.box_b;
   p.nfull = pl.nfull;
