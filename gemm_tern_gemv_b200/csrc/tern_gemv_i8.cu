@@ -253,11 +253,12 @@ __global__ void __launch_bounds__((i8_max_nw(CPS) + 1) * 32, CPS)
   const uint32_t empty0 = full0 + 8u * (uint32_t)p.stages;
   int* ctl = reinterpret_cast<int*>(smem + (size_t)p.stages * p.stage_bytes + 16 * p.stages);  // [0] abort, [1..] S_b
   volatile int* abort_flag = ctl;
-  int* Xs = ctl + 8;  // [BATCH][xk]: X = round(x * 2^S) of the CTA's activations, zero past K
-  uint4* frag = reinterpret_cast<uint4*>(Xs + BATCH * p.xk);
+  uint4* frag = reinterpret_cast<uint4*>(ctl + 8);
   float* red = reinterpret_cast<float*>(frag + (size_t)p.L * kMP * BATCH * kEnt);  // [32][BATCH]; Q1: + corr
   float* corr = red + 32 * BATCH;                                                      // Q1: [L][2][BATCH]
-  float* part = corr + (LAYOUT == TERN_Q1_0_G128 ? p.L * 2 * BATCH : 0);               // [tmax][NW][BATCH][16]
+  // the partial sums of the main loop share their space with X, which only the prologue uses
+  float* part = corr + (LAYOUT == TERN_Q1_0_G128 ? (p.L * 2 * BATCH + 3) / 4 * 4 : 0);  // [tmax][NW][BATCH][16], 16-B aligned
+  int* Xs = reinterpret_cast<int*>(part);  // [BATCH][xk]: X = round(x * 2^S) of the CTA's activations, zero past K
 
   // work: cluster c owns tiles [t0, t1); CTA rank r of the cluster owns K slice r (units [u0, u1))
   const int KS = (int)cluster_size();
@@ -599,7 +600,9 @@ __global__ void __launch_bounds__((i8_max_nw(CPS) + 1) * 32, CPS)
         ub = ck ? ue : 0;
         ue = chunk_lo(ck + 1);
       }
-      if (!mbar_wait(full0 + 8u * s, ph, abort_flag, p.status, p.wait_ns)) break;
+      // every lane waits (each must observe the copy's completion); the verdict is made warp-uniform,
+      // so that a lane whose wait ran out cannot leave the others stuck in the shuffles below
+      if (!__all_sync(0xffffffffu, mbar_wait(full0 + 8u * s, ph, abort_flag, p.status, p.wait_ns))) break;
       float acc[BATCH][2];
 #pragma unroll
       for (int b = 0; b < BATCH; b++) acc[b][0] = acc[b][1] = 0.f;
@@ -774,11 +777,10 @@ size_t i8_smem_bytes(const I8Params& p, int batch) {
   using T = I8L<LAYOUT>;
   size_t s = 1024;  // alignment slack
   s += (size_t)p.stages * p.stage_bytes + 16 * (size_t)p.stages + 32;
-  s += 4 * (size_t)batch * p.xk;
   s += (size_t)p.L * T::kMP * batch * T::kEnt * 16;
   s += 4 * 32 * (size_t)batch;
-  if (LAYOUT == TERN_Q1_0_G128) s += 4 * (size_t)p.L * 2 * batch;
-  s += 4 * (size_t)p.tmax * p.nw * batch * 16;
+  if (LAYOUT == TERN_Q1_0_G128) s += 4 * (((size_t)p.L * 2 * batch + 3) / 4 * 4);
+  s += std::max(4 * (size_t)p.tmax * p.nw * batch * 16, 4 * (size_t)batch * p.xk);  // partials / X (disjoint in time)
   return s;
 }
 
@@ -790,7 +792,9 @@ const void* i8_kernel() {
 }  // namespace
 
 // Plan for `cps` CTAs per SM; ok = false when nothing fits.
-static I8Plan i8_plan_cps(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms, int cps) {
+// Plan for exactly `cps` CTAs per SM, a K split over `ks` CTAs of a cluster and `nw` consumer warps
+// (fewer when a slice has fewer units); ok = false when it does not fit.
+static I8Plan i8_plan_cfg(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms, int cps, int ks, int nw) {
   if (batch < 1 || batch > 2) return I8Plan{};
   const int unit_k = layout == TERN_T3_5PB_G128 ? 160 : 256;
   const int unit_b = layout == TERN_Q2_0_G128 ? 64 : 32;
@@ -799,72 +803,89 @@ static I8Plan i8_plan_cps(int32_t layout, int64_t n, int64_t k, int64_t batch, i
   // whole units only (Q2_0_g128 and Q1_0_g128: K a multiple of 256); other shapes use the older kernels
   if (rb <= 0 || rb % unit_b || n > (int64_t)INT32_MAX) return I8Plan{};
   const int units = (int)(rb / unit_b);
-  const int tiles = (int)((n + 15) / 16);
-  const int groups = (int)(k / kGroup);
-  const size_t cap = (size_t)(228 / cps - 1) * 1024;
-  I8Plan best{};
-  double best_cost = 1e300;
-  // cost of a K split ks: tiles per cluster x units per warp, fewer than 16 warps counted as slower
-  for (int ks : {1, 2, 4}) {
-    const int L = (units + ks - 1) / ks;
-    if (ks > 1 && L < 8) continue;
-    I8Plan pl{};
-    pl.ks = ks;
-    pl.L = L;
-    pl.units = units;
-    pl.tiles = tiles;
-    pl.groups = groups;
-    const int slice_b = L * unit_b;
-    pl.box_b = std::min(1024, slice_b);
-    pl.nfull = slice_b / pl.box_b;
-    pl.rem_b = slice_b - pl.nfull * pl.box_b;
-    // scale box: from the first slice group rounded down to 8, wide enough for every slice
-    int scw = 8;
-    for (int r = 0; r < ks; r++) {
-      const int ua = r * L, ue = std::min(units, ua + L);
-      if (ua >= ue) continue;
-      const int g0 = ua * unit_k / kGroup, g1 = std::min(groups, (ue * unit_k + kGroup - 1) / kGroup);
-      scw = std::max(scw, g1 - (g0 & ~7));
-    }
-    pl.sc_w = (scw + 7) / 8 * 8;
-    if (pl.sc_w > 256) continue;
-    pl.code_bytes = 16 * slice_b;
-    pl.stage_bytes = (pl.code_bytes + 16 * pl.sc_w * 2 + 1023) / 1024 * 1024;
-    pl.xk = (L * unit_k + 7) / 8 * 8;
-    const int clusters = std::max(1, cps * sms / ks);
-    pl.tmax = (tiles + clusters - 1) / clusters;
-    for (int nw = std::min(L, 8); nw <= std::min(L, i8_max_nw(cps)); nw++) {
-      if (pl.xk > kXV * 8 * (nw + 1) * 32) continue;  // every activation of the slice converted in one pass
-      const size_t fixed = 1024 + 48 + 4 * (size_t)batch * pl.xk + (size_t)L * ent_bytes * batch + 128 * (size_t)batch +
-                           (layout == TERN_Q1_0_G128 ? 8 * (size_t)L * batch : 0) + 64 * (size_t)pl.tmax * nw * batch;
-      if (fixed + 2 * (size_t)(pl.stage_bytes + 16) > cap) continue;
-      // the slowest warp sets the tile time; an SM streams faster the more warps it has (measured: 16
-      // warps with one or two units each beat 13 warps with two each), so fewer warps count as slower
-      const int per_warp = (L + nw - 1) / nw;
-      const double cost = (double)pl.tmax * per_warp * (16.0 / std::min(16, cps * nw)) * (1.0 + 0.02 * (ks - 1)) +
-                          0.001 * std::abs(cps * nw - 16);
-      if (cost < best_cost) {
-        best_cost = cost;
-        best = pl;
-        best.nw = nw;
-        best.npr = (L % nw == 0 && L / nw == 1) ? 1 : 0;
-        best.stages = (int)std::min<size_t>(8, (cap - fixed) / (pl.stage_bytes + 16));
-        best.ok = true;
-        best.cps = cps;
-      }
-    }
+  const int L = (units + ks - 1) / ks;
+  if (ks > 1 && L < 8) return I8Plan{};
+  nw = std::min(nw, L);
+  if (nw < 1 || nw > i8_max_nw(cps)) return I8Plan{};
+  I8Plan pl{};
+  pl.ks = ks;
+  pl.L = L;
+  pl.units = units;
+  pl.tiles = (int)((n + 15) / 16);
+  pl.groups = (int)(k / kGroup);
+  const int slice_b = L * unit_b;
+  pl.box_b = std::min(1024, slice_b);
+  pl.nfull = slice_b / pl.box_b;
+  pl.rem_b = slice_b - pl.nfull * pl.box_b;
+  // scale box: from the first slice group rounded down to 8, wide enough for every slice
+  int scw = 8;
+  for (int r = 0; r < ks; r++) {
+    const int ua = r * L, ue = std::min(units, ua + L);
+    if (ua >= ue) continue;
+    const int g0 = ua * unit_k / kGroup, g1 = std::min(pl.groups, (ue * unit_k + kGroup - 1) / kGroup);
+    scw = std::max(scw, g1 - (g0 & ~7));
   }
-  return best;
+  pl.sc_w = (scw + 7) / 8 * 8;
+  if (pl.sc_w > 256) return I8Plan{};
+  pl.code_bytes = 16 * slice_b;
+  pl.stage_bytes = (pl.code_bytes + 16 * pl.sc_w * 2 + 1023) / 1024 * 1024;
+  pl.xk = (L * unit_k + 7) / 8 * 8;
+  if (pl.xk > kXV * 8 * (nw + 1) * 32) return I8Plan{};  // every activation of the slice converted in one pass
+  const int clusters = std::max(1, cps * sms / ks);
+  pl.tmax = (pl.tiles + clusters - 1) / clusters;
+  const size_t cap = (size_t)(228 / cps - 1) * 1024;
+  const size_t fixed = 1024 + 48 + (size_t)L * ent_bytes * batch + 128 * (size_t)batch +
+                       (layout == TERN_Q1_0_G128 ? 4 * (((size_t)L * 2 * batch + 3) / 4 * 4) : 0) +
+                       std::max(64 * (size_t)pl.tmax * nw * batch, 4 * (size_t)batch * pl.xk);
+  if (fixed + 2 * (size_t)(pl.stage_bytes + 16) > cap) return I8Plan{};
+  pl.nw = nw;
+  pl.npr = (L % nw == 0 && L / nw == 1) ? 1 : 0;
+  pl.stages = (int)std::min<size_t>(8, (cap - fixed) / (pl.stage_bytes + 16));
+  pl.cps = cps;
+  pl.ok = true;
+  return pl;
 }
 
 // Plan of the int8 kernel for (layout, n, k, batch) on `sms` SMs; ok = false when it does not apply.
-// Two CTAs per SM when one per SM would give each SM at least 14 row tiles or split K over a cluster
-// (measured: the LM head and the 27B-class matrices gain 10-20 %, the 8B-class ones lose).
+// The rule comes from a sweep of every (CTAs per SM, K split, warps) on B200 at batch 1 with weights
+// streamed from HBM: one K slice whenever the slice fits; then two CTAs of 8 consumer warps per SM
+// once one CTA per SM would own at least 14 row tiles (LM head, 27B-class layers: 2-10 % faster),
+// otherwise one CTA of 16 warps, or of 8 when it owns at most two tiles (4096 x 4096: 7-9 %); a slice
+// that does not fit is split over a pair of CTAs at one CTA of 12 warps per SM (K = 12288 / 17408:
+// 30-35 % faster than four CTAs at two per SM). A split over four is never faster; it stays as the
+// last resort before the older kernels.
 I8Plan i8_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
-  const I8Plan one = i8_plan_cps(layout, n, k, batch, sms, 1);
-  if (one.ok && one.tmax < 14 && one.ks == 1) return one;
-  const I8Plan two = i8_plan_cps(layout, n, k, batch, sms, 2);
-  return two.ok ? two : one;
+  const I8Plan one = i8_plan_cfg(layout, n, k, batch, sms, 1, 1, 16);
+  if (one.ok) {
+    if (one.tmax >= 14) {
+      const I8Plan two = i8_plan_cfg(layout, n, k, batch, sms, 2, 1, 8);
+      if (two.ok) return two;
+    }
+    if (one.tmax <= 2) {
+      const I8Plan few = i8_plan_cfg(layout, n, k, batch, sms, 1, 1, 8);
+      if (few.ok) return few;
+    }
+    return one;
+  }
+  // one slice with the most warps the pass over x allows (a slice too long for 16 warps' threads)
+  const I8Plan wide = i8_plan_cfg(layout, n, k, batch, sms, 1, 1, kI8MaxNW1);
+  if (wide.ok) return wide;
+  // two rows of x with a K split and >= 32 tiles per cluster keep a partial sum per tile, which leaves
+  // room for two ring stages only: the older kernels are faster there (LM head, batch 2: 84 vs 95 us)
+  if (batch == 2) {
+    const int tiles = (int)((n + 15) / 16), tmax2 = (tiles + sms / 2 - 1) / (sms / 2);
+    if (tmax2 >= 32) return I8Plan{};
+  }
+  for (int nw : {12, 16, 8, kI8MaxNW1, 10, 6, 4}) {
+    const I8Plan pair = i8_plan_cfg(layout, n, k, batch, sms, 1, 2, nw);
+    if (pair.ok) return pair;
+  }
+  for (int cps : {2, 1})
+    for (int nw : {8, 16, kI8MaxNW1, 12, 6, 4}) {
+      const I8Plan four = i8_plan_cfg(layout, n, k, batch, sms, cps, 4, nw);
+      if (four.ok) return four;
+    }
+  return I8Plan{};
 }
 
 namespace {
