@@ -1119,7 +1119,6 @@ __global__ void __launch_bounds__(NW * 32, CPS)
             dst[2 * rt + 1] = acc[rt][1];
           }
         }
-        s_store<LAYOUT, RT>(a, c_tile, -1, lane, acc);
       } else {
         const int seg = wi - (c_tile * nwin) / a.run;
         s_store<LAYOUT, RT>(a, c_tile, split * a.kmax + seg, lane, acc);

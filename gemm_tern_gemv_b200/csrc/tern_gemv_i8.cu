@@ -34,7 +34,6 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
-#include <mutex>
 
 #include "sm100.cuh"
 #include "tern_internal.cuh"
