@@ -246,9 +246,10 @@ TERN_API tern_status tern_gemv_opt(const tern_matrix* W, const uint16_t* x, int6
  *   - Every call on a device shares the one array: calls that overlap on the GPU (different
  *     streams without ordering between them) race and give wrong results. Order them.
  *   - A matrix / batch whose split-K workspace (tern_gemv_workspace_bytes) exceeds
- *     TERN_GEMV_NOALLOC_SCRATCH_BYTES returns TERN_ERR_WORKSPACE before any launch; batch <= 8
- *     fits for N <= 151936 at K = 4096 and for N <= 34816 up to K = 17408, and batches of 17 or
- *     more with N % 8 == 0 need no scratch.
+ *     TERN_GEMV_NOALLOC_SCRATCH_BYTES returns TERN_ERR_WORKSPACE before any launch. Checked on the
+ *     host for a 148-SM B200 (the plan depends on the SM count): batch <= 8 fits for N <= 151936 at
+ *     K = 4096 and for N <= 34816 up to K = 17408, and batches of 17 or more with N % 8 == 0 need
+ *     no scratch.
  * Errors: those of tern_gemv, TERN_ERR_WORKSPACE as above, TERN_ERR_CUDA if the address lookup
  * or the memset fails. */
 TERN_API tern_status tern_gemv_noalloc(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y,
