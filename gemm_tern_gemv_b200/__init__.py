@@ -36,7 +36,8 @@ class TernError(RuntimeError):
 
 
 class TernGemvOptsC(ctypes.Structure):
-    _fields_ = [("flags", ctypes.c_uint32), ("device_status", ctypes.c_void_p), ("wait_limit_ns", ctypes.c_uint64)]
+    _fields_ = [("flags", ctypes.c_uint32), ("device_status", ctypes.c_void_p), ("wait_limit_ns", ctypes.c_uint64),
+                ("rotate_signs", ctypes.c_void_p)]
 
 
 class TernMatrixC(ctypes.Structure):
@@ -63,6 +64,8 @@ SIGNATURES = {
                                     ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint32, ctypes.c_void_p]),
     "tern_gemv_opt": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                      ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(TernGemvOptsC), ctypes.c_void_p]),
+    "tern_gemv_opt_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(TernMatrixC), ctypes.c_int64,
+                                                        ctypes.POINTER(TernGemvOptsC)]),
     "tern_gemv_noalloc": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                          ctypes.c_void_p]),
     "tern_gemm": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
@@ -280,10 +283,23 @@ def gemv(W: TernMatrix, x, y=None, workspace=None, static_weights: bool = False)
     return y
 
 
+def _opts(static_weights=False, status=None, wait_limit_ns=0, rotate_signs=None):
+    return TernGemvOptsC(GEMV_STATIC_WEIGHTS if static_weights else 0, _ptr(status) if status is not None else None,
+                         int(wait_limit_ns), _ptr(rotate_signs) if rotate_signs is not None else None)
+
+
+def gemv_opt_workspace_bytes(W: TernMatrix, batch: int, rotate_signs=None) -> int:
+    """tern_gemv_opt_workspace_bytes for these options (only the rotation changes the size)."""
+    c = W.c()
+    o = _opts(rotate_signs=rotate_signs)
+    return int(lib().tern_gemv_opt_workspace_bytes(ctypes.byref(c), batch, ctypes.byref(o)))
+
+
 def gemv_opt(W: TernMatrix, x, y=None, workspace=None, static_weights: bool = False, status=None,
-             wait_limit_ns: int = 0):
+             wait_limit_ns: int = 0, rotate_signs=None):
     """tern_gemv_opt: gemv with an optional device status word (uint32 tensor, TERN_DEVICE_TIMEOUT is
-    OR-ed in when a pipeline wait runs out) and a bound on each wait (0 = the library default)."""
+    OR-ed in when a pipeline wait runs out), a bound on each wait (0 = the library default) and an
+    optional block Hadamard rotation of x (int8 tensor of 1024 signs: y = W (R x))."""
     torch = _torch()
     if x.dim() == 1:
         x = x.unsqueeze(0)
@@ -292,11 +308,11 @@ def gemv_opt(W: TernMatrix, x, y=None, workspace=None, static_weights: bool = Fa
     if y is None:
         y = torch.empty((batch, W.n), dtype=torch.float16, device=x.device)
     if workspace is None:
-        workspace = gemv_workspace(W, batch)
+        nb = gemv_opt_workspace_bytes(W, batch, rotate_signs)
+        workspace = torch.zeros(nb, dtype=torch.uint8, device=W.codes.device) if nb else None
     wsb = workspace.numel() if workspace is not None else 0
     c = W.c()
-    o = TernGemvOptsC(GEMV_STATIC_WEIGHTS if static_weights else 0, _ptr(status) if status is not None else None,
-                      int(wait_limit_ns))
+    o = _opts(static_weights, status, wait_limit_ns, rotate_signs)
     st = lib().tern_gemv_opt(ctypes.byref(c), _ptr(x), batch, _ptr(y), _ptr(workspace), wsb, ctypes.byref(o),
                              _stream_handle())
     _check(st, "tern_gemv_opt")

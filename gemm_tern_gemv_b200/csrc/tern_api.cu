@@ -5,6 +5,7 @@
 #include <mutex>
 #include <vector>
 
+#include "tern_fwht.cuh"
 #include "tern_internal.cuh"
 
 namespace tern {
@@ -146,25 +147,68 @@ tern_status tern_gemv_ex(const tern_matrix* W, const uint16_t* x, int64_t batch,
   return tern_gemv_opt(W, x, batch, y, workspace, workspace_bytes, &o, stream);
 }
 
+// The plan of tern_gemv_opt: the GEMV plan, and whether x is rotated inside the int8-plane kernel (same
+// work split as without the rotation) or first into the workspace at rot_off.
+struct OptPlan {
+  GemvPlan plan;
+  bool fused;
+  size_t rot_off, ws;
+};
+static OptPlan opt_plan(const tern_matrix& W, int64_t batch, bool rotate) {
+  OptPlan o{};
+  o.plan = gemv_plan(W.layout, W.n, W.k, batch, sm_count());
+  o.ws = o.plan.ws_bytes;
+  if (rotate) {
+    if (o.plan.i8) {
+      const I8Plan r = i8_plan_rotate(o.plan.i8p, W.layout, W.n, W.k, std::min<int64_t>(batch, 2), sm_count());
+      if (r.ok) {
+        o.plan.i8p = r;
+        o.fused = true;
+        return o;
+      }
+    }
+    o.rot_off = (o.ws + 255) / 256 * 256;
+    o.ws = o.rot_off + (size_t)batch * (size_t)W.k * 2;
+  }
+  return o;
+}
+
+size_t tern_gemv_opt_workspace_bytes(const tern_matrix* W, int64_t batch, const tern_gemv_opts* opts) {
+  const bool rotate = opts && opts->rotate_signs;
+  if (!rotate) return tern_gemv_workspace_bytes(W, batch);
+  if (!W || W->n <= 0 || W->k <= 0 || W->k % kRotBlock) return 0;
+  if (!valid_layout(W->layout)) return 0;
+  if (batch < 1 || batch > TERN_GEMV_MAX_BATCH) return 0;
+  return opt_plan(*W, batch, true).ws;
+}
+
 tern_status tern_gemv_opt(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y, void* workspace,
                           size_t workspace_bytes, const tern_gemv_opts* opts, void* stream) {
   const uint32_t flags = opts ? opts->flags : 0u;
   uint32_t* status = opts ? opts->device_status : nullptr;
   const uint64_t wait_ns = opts ? opts->wait_limit_ns : 0u;
+  const int8_t* signs = opts ? opts->rotate_signs : nullptr;
   if (flags & ~(uint32_t)TERN_GEMV_STATIC_WEIGHTS) return TERN_ERR_INVALID_ARG;
   if (status && (reinterpret_cast<uintptr_t>(status) & 3u)) return TERN_ERR_ALIGNMENT;
   tern_status s = check_matrix(W);
   if (s != TERN_OK) return s;
   if (batch < 1 || batch > TERN_GEMV_MAX_BATCH || !x || !y) return TERN_ERR_INVALID_ARG;
+  if (signs && W->k % kRotBlock) return TERN_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y)) return TERN_ERR_ALIGNMENT;
   if (!gemv_supported(W->layout, W->n, W->k, batch)) return TERN_ERR_UNSUPPORTED;
-  GemvPlan plan = gemv_plan(W->layout, W->n, W->k, batch, sm_count());
-  if (plan.ws_bytes) {
-    if (!workspace || workspace_bytes < plan.ws_bytes) return TERN_ERR_WORKSPACE;
+  const OptPlan op = opt_plan(*W, batch, signs != nullptr);
+  if (op.ws) {
+    if (!workspace || workspace_bytes < op.ws) return TERN_ERR_WORKSPACE;
     if (!aligned16(workspace)) return TERN_ERR_ALIGNMENT;
   }
-  return from_cuda(launch_gemv(*W, x, (int)batch, y, workspace, plan, static_cast<cudaStream_t>(stream), flags,
-                               status, wait_ns));
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (signs && !op.fused) {
+    uint16_t* xr = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + op.rot_off);
+    const cudaError_t e = launch_rotate(x, batch, W->k, signs, xr, st);
+    if (e != cudaSuccess) return from_cuda(e);
+    return from_cuda(launch_gemv(*W, xr, (int)batch, y, workspace, op.plan, st, flags, status, wait_ns));
+  }
+  return from_cuda(launch_gemv(*W, x, (int)batch, y, workspace, op.plan, st, flags, status, wait_ns, signs));
 }
 
 tern_status tern_gemv_noalloc(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y, void* stream) {

@@ -1440,16 +1440,18 @@ GemvPlan gemv_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms)
 }
 
 cudaError_t launch_gemv(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y, void* workspace,
-                        const GemvPlan& plan, cudaStream_t st, uint32_t flags, uint32_t* status, uint64_t wait_ns) {
+                        const GemvPlan& plan, cudaStream_t st, uint32_t flags, uint32_t* status, uint64_t wait_ns,
+                        const int8_t* signs) {
   if (plan.i8) {
     // one launch per pair of rows of x, in order on the stream (binary batches 3-4)
     for (int b0 = 0; b0 < batch; b0 += 2) {
       const cudaError_t e = launch_gemv_i8(W, x + (int64_t)b0 * W.k, std::min(2, batch - b0), y + (int64_t)b0 * W.n,
-                                           plan.i8p, st, flags, status, wait_ns);
+                                           plan.i8p, st, flags, status, wait_ns, signs);
       if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
   }
+  if (signs) return cudaErrorInvalidValue;  // only the int8-plane kernel rotates x itself
   if (plan.gemm) return launch_gemm(W, x, batch, y, status, st);
   Args a;
   a.codes = static_cast<const uint8_t*>(W.codes);

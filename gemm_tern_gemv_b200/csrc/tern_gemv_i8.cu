@@ -36,6 +36,7 @@
 #include <algorithm>
 
 #include "sm100.cuh"
+#include "tern_fwht.cuh"
 #include "tern_internal.cuh"
 
 namespace tern {
@@ -75,6 +76,9 @@ struct I8Params {
   int stage_bytes, code_bytes, stages;
   int tmax;           // largest number of tiles a cluster owns
   int xk;             // activations held per CTA (halves, multiple of 8)
+  const int8_t* signs;  // non-null: multiply by R x (block Hadamard rotation of x, done in the prologue)
+  int rot_off;        // rotated x: byte offset within the partial-sum space (past X and the FWHT scratch)
+  int rot_bytes;      // bytes of that space the rotation needs
 };
 
 // ---- small device helpers --------------------------------------------------------------------------
@@ -310,6 +314,39 @@ __global__ void __launch_bounds__((i8_max_nw(CPS) + 1) * 32, CPS)
 
   // ---- activations: x -> int8 planes in B-fragment order -----------------------------------------
   const int xend = min(p.k, u1 * T::kUnitK);  // activations past K (base-3 padding) read as zero
+  // the activations the fragments are built from: x itself, or R x for the 1024-blocks that cover this
+  // CTA's slice, rotated here into shared memory by groups of 128 threads (the same transform and fp16
+  // rounding as tern_hadamard_rotate, so the product equals W applied to that kernel's output)
+  const uint16_t* xsrc = p.x;
+  int64_t xsrc_stride = p.k;
+  int xsrc_off = 0;
+  if (p.signs) {
+    const int blk0 = kx0 / kRotBlock, nb = (xend + kRotBlock - 1) / kRotBlock - blk0;
+    uint16_t* xr = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(part) + p.rot_off);  // [BATCH][nb * 1024]
+    float* fsh = part;  // [groups][1024] floats: the FWHT exchange buffer (X is written only afterwards)
+    const int groups = min((int)blockDim.x / kRotThreads, 4), grp = tid / kRotThreads, t = tid % kRotThreads;
+    if (grp < groups) {
+      for (int it = grp; it < BATCH * nb; it += groups) {
+        const int b = it / nb, j = it % nb;
+        const uint16_t* src = p.x + (int64_t)b * p.k + (int64_t)(blk0 + j) * kRotBlock;
+        float v[8];
+#pragma unroll
+        for (int r = 0; r < 8; r++) {
+          const int i = t + kRotThreads * r;
+          const float xv = __half2float(__ushort_as_half(src[i]));
+          v[r] = p.signs[i] < 0 ? -xv : xv;
+        }
+        fwht1024(v, fsh + grp * kRotBlock, t, SyncGroup128{grp + 1});
+#pragma unroll
+        for (int r = 0; r < 8; r++)
+          xr[b * nb * kRotBlock + j * kRotBlock + t + kRotThreads * r] = __half_as_ushort(__float2half_rn(v[r] * 0.03125f));
+      }
+    }
+    __syncthreads();
+    xsrc = xr;
+    xsrc_stride = (int64_t)nb * kRotBlock;
+    xsrc_off = blk0 * kRotBlock;
+  }
   // pass 1: each thread loads up to kXV vectors of 8 activations per row of x, the CTA takes max|x|,
   // and every activation is converted once to X = round(x * 2^S) (exact for S = 24)
   uint4 xv[BATCH][kXV];
@@ -322,10 +359,11 @@ __global__ void __launch_bounds__((i8_max_nw(CPS) + 1) * 32, CPS)
       const int kk = kx0 + e;
       if (e < p.xk) {
         if (kk + 8 <= xend) {
-          v = *reinterpret_cast<const uint4*>(p.x + (int64_t)b * p.k + kk);
+          v = *reinterpret_cast<const uint4*>(xsrc + (int64_t)b * xsrc_stride + (kk - xsrc_off));
         } else if (kk < xend) {
           uint16_t h[8];
-          for (int jj = 0; jj < 8; jj++) h[jj] = (kk + jj < xend) ? p.x[(int64_t)b * p.k + kk + jj] : (uint16_t)0;
+          for (int jj = 0; jj < 8; jj++)
+            h[jj] = (kk + jj < xend) ? xsrc[(int64_t)b * xsrc_stride + (kk + jj - xsrc_off)] : (uint16_t)0;
           v = make_uint4(h[0] | (uint32_t)h[1] << 16, h[2] | (uint32_t)h[3] << 16, h[4] | (uint32_t)h[5] << 16,
                          h[6] | (uint32_t)h[7] << 16);
         }
@@ -779,7 +817,8 @@ size_t i8_smem_bytes(const I8Params& p, int batch) {
   s += (size_t)p.L * T::kMP * batch * T::kEnt * 16;
   s += 4 * 32 * (size_t)batch;
   if (LAYOUT == TERN_Q1_0_G128) s += 4 * (((size_t)p.L * 2 * batch + 3) / 4 * 4);
-  s += std::max(4 * (size_t)p.tmax * p.nw * batch * 16, 4 * (size_t)batch * p.xk);  // partials / X (disjoint in time)
+  // partials / X / the rotated x (disjoint in time)
+  s += std::max({4 * (size_t)p.tmax * p.nw * batch * 16, 4 * (size_t)batch * p.xk, (size_t)p.rot_bytes});
   return s;
 }
 
@@ -793,7 +832,8 @@ const void* i8_kernel() {
 // Plan for `cps` CTAs per SM; ok = false when nothing fits.
 // Plan for exactly `cps` CTAs per SM, a K split over `ks` CTAs of a cluster and `nw` consumer warps
 // (fewer when a slice has fewer units); ok = false when it does not fit.
-static I8Plan i8_plan_cfg(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms, int cps, int ks, int nw) {
+static I8Plan i8_plan_cfg(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms, int cps, int ks, int nw,
+                          bool rotate = false) {
   if (batch < 1 || batch > 2) return I8Plan{};
   const int unit_k = layout == TERN_T3_5PB_G128 ? 160 : 256;
   const int unit_b = layout == TERN_Q2_0_G128 ? 64 : 32;
@@ -832,10 +872,23 @@ static I8Plan i8_plan_cfg(int32_t layout, int64_t n, int64_t k, int64_t batch, i
   if (pl.xk > kXV * 8 * (nw + 1) * 32) return I8Plan{};  // every activation of the slice converted in one pass
   const int clusters = std::max(1, cps * sms / ks);
   pl.tmax = (pl.tiles + clusters - 1) / clusters;
+  if (rotate) {
+    // groups of 128 threads rotate the 1024-blocks covering the slice: exchange buffers of 4 KB per
+    // group (sharing space with X), then the rotated fp16 activations of every covering block
+    const int groups = std::min((nw + 1) * 32 / kRotThreads, 4);
+    if (k % kRotBlock || groups < 1) return I8Plan{};
+    int64_t cover = 0;
+    for (int r = 0; r < ks; r++) {
+      const int64_t a = (int64_t)r * L * unit_k, e = std::min<int64_t>(k, (int64_t)(r + 1) * L * unit_k);
+      if (a < e) cover = std::max(cover, ((e + kRotBlock - 1) / kRotBlock - a / kRotBlock) * kRotBlock);
+    }
+    pl.rot_off = (int)((std::max<size_t>(4 * (size_t)batch * pl.xk, (size_t)groups * kRotBlock * 4) + 15) / 16 * 16);
+    pl.rot_bytes = pl.rot_off + (int)(2 * batch * cover);
+  }
   const size_t cap = (size_t)(228 / cps - 1) * 1024;
   const size_t fixed = 1024 + 48 + (size_t)L * ent_bytes * batch + 128 * (size_t)batch +
                        (layout == TERN_Q1_0_G128 ? 4 * (((size_t)L * 2 * batch + 3) / 4 * 4) : 0) +
-                       std::max(64 * (size_t)pl.tmax * nw * batch, 4 * (size_t)batch * pl.xk);
+                       std::max({64 * (size_t)pl.tmax * nw * batch, 4 * (size_t)batch * pl.xk, (size_t)pl.rot_bytes});
   if (fixed + 2 * (size_t)(pl.stage_bytes + 16) > cap) return I8Plan{};
   pl.nw = nw;
   pl.npr = (L % nw == 0 && L / nw == 1) ? 1 : 0;
@@ -853,6 +906,14 @@ static I8Plan i8_plan_cfg(int32_t layout, int64_t n, int64_t k, int64_t batch, i
 // that does not fit is split over a pair of CTAs at one CTA of 12 warps per SM (K = 12288 / 17408:
 // 30-35 % faster than four CTAs at two per SM). A split over four is never faster; it stays as the
 // last resort before the older kernels.
+// The same CTA shape and work split as `base` (so the same sums in the same order) with room for the
+// block Hadamard rotation of x in the prologue; ok = false when it does not fit.
+I8Plan i8_plan_rotate(const I8Plan& base, int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
+  if (!base.ok) return I8Plan{};
+  const I8Plan r = i8_plan_cfg(layout, n, k, batch, sms, base.cps, base.ks, base.nw, true);
+  return (r.ok && r.nw == base.nw && r.L == base.L && r.tmax == base.tmax) ? r : I8Plan{};
+}
+
 I8Plan i8_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms) {
   const I8Plan one = i8_plan_cfg(layout, n, k, batch, sms, 1, 1, 16);
   if (one.ok) {
@@ -891,7 +952,7 @@ namespace {
 
 template <int LAYOUT, int BATCH, int NPR, int CPS>
 cudaError_t launch_i8_t(const tern_matrix& W, const uint16_t* x, uint16_t* y, const I8Plan& pl, cudaStream_t st,
-                        uint32_t flags, uint32_t* status, uint64_t wait_ns) {
+                        uint32_t flags, uint32_t* status, uint64_t wait_ns, const int8_t* signs) {
   using T = I8L<LAYOUT>;
   I8Params p{};
   p.x = x;
@@ -920,6 +981,10 @@ cudaError_t launch_i8_t(const tern_matrix& W, const uint16_t* x, uint16_t* y, co
   p.stages = pl.stages;
   p.tmax = pl.tmax;
   p.xk = pl.xk;
+  p.signs = signs;
+  p.rot_off = signs ? pl.rot_off : 0;
+  p.rot_bytes = signs ? pl.rot_bytes : 0;
+  if (signs && !pl.rot_bytes) return cudaErrorInvalidValue;  // the plan has no room for the rotation
   const size_t smem = i8_smem_bytes<LAYOUT>(p, BATCH);
   const void* kern = i8_kernel<LAYOUT, BATCH, NPR, CPS>();
   // the planned grid: clusters own disjoint tiles and never wait on one another, so clusters that
@@ -969,27 +1034,27 @@ cudaError_t launch_i8_t(const tern_matrix& W, const uint16_t* x, uint16_t* y, co
 
 template <int LAYOUT, int CPS>
 cudaError_t launch_i8_c(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y, const I8Plan& pl,
-                        cudaStream_t st, uint32_t flags, uint32_t* status, uint64_t wait_ns) {
+                        cudaStream_t st, uint32_t flags, uint32_t* status, uint64_t wait_ns, const int8_t* signs) {
   if (batch == 1)
-    return pl.npr ? launch_i8_t<LAYOUT, 1, 1, CPS>(W, x, y, pl, st, flags, status, wait_ns)
-                  : launch_i8_t<LAYOUT, 1, 0, CPS>(W, x, y, pl, st, flags, status, wait_ns);
-  return pl.npr ? launch_i8_t<LAYOUT, 2, 1, CPS>(W, x, y, pl, st, flags, status, wait_ns)
-                : launch_i8_t<LAYOUT, 2, 0, CPS>(W, x, y, pl, st, flags, status, wait_ns);
+    return pl.npr ? launch_i8_t<LAYOUT, 1, 1, CPS>(W, x, y, pl, st, flags, status, wait_ns, signs)
+                  : launch_i8_t<LAYOUT, 1, 0, CPS>(W, x, y, pl, st, flags, status, wait_ns, signs);
+  return pl.npr ? launch_i8_t<LAYOUT, 2, 1, CPS>(W, x, y, pl, st, flags, status, wait_ns, signs)
+                : launch_i8_t<LAYOUT, 2, 0, CPS>(W, x, y, pl, st, flags, status, wait_ns, signs);
 }
 template <int LAYOUT>
 cudaError_t launch_i8_l(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y, const I8Plan& pl,
-                        cudaStream_t st, uint32_t flags, uint32_t* status, uint64_t wait_ns) {
-  return pl.cps == 2 ? launch_i8_c<LAYOUT, 2>(W, x, batch, y, pl, st, flags, status, wait_ns)
-                     : launch_i8_c<LAYOUT, 1>(W, x, batch, y, pl, st, flags, status, wait_ns);
+                        cudaStream_t st, uint32_t flags, uint32_t* status, uint64_t wait_ns, const int8_t* signs) {
+  return pl.cps == 2 ? launch_i8_c<LAYOUT, 2>(W, x, batch, y, pl, st, flags, status, wait_ns, signs)
+                     : launch_i8_c<LAYOUT, 1>(W, x, batch, y, pl, st, flags, status, wait_ns, signs);
 }
 
 }  // namespace
 
 cudaError_t launch_gemv_i8(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y, const I8Plan& pl,
-                           cudaStream_t st, uint32_t flags, uint32_t* status, uint64_t wait_ns) {
-  if (W.layout == TERN_Q2_0_G128) return launch_i8_l<TERN_Q2_0_G128>(W, x, batch, y, pl, st, flags, status, wait_ns);
-  if (W.layout == TERN_Q1_0_G128) return launch_i8_l<TERN_Q1_0_G128>(W, x, batch, y, pl, st, flags, status, wait_ns);
-  return launch_i8_l<TERN_T3_5PB_G128>(W, x, batch, y, pl, st, flags, status, wait_ns);
+                           cudaStream_t st, uint32_t flags, uint32_t* status, uint64_t wait_ns, const int8_t* signs) {
+  if (W.layout == TERN_Q2_0_G128) return launch_i8_l<TERN_Q2_0_G128>(W, x, batch, y, pl, st, flags, status, wait_ns, signs);
+  if (W.layout == TERN_Q1_0_G128) return launch_i8_l<TERN_Q1_0_G128>(W, x, batch, y, pl, st, flags, status, wait_ns, signs);
+  return launch_i8_l<TERN_T3_5PB_G128>(W, x, batch, y, pl, st, flags, status, wait_ns, signs);
 }
 
 }  // namespace tern

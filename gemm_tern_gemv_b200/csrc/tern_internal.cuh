@@ -47,11 +47,16 @@ struct I8Plan {
   int xk;          // activations per CTA (halves)
   int tmax;        // tiles per cluster (upper bound)
   int cps;         // CTAs per SM (1 or 2)
+  int rot_off, rot_bytes;  // block Hadamard rotation of x in the prologue (0 = no room planned)
 };
 I8Plan i8_plan(int32_t layout, int64_t n, int64_t k, int64_t batch, int sms);
-// status / wait_ns: optional device status word and bound on each pipeline wait (0 = 1 s)
+// `base` with room for rotating x in the prologue, same work split; ok = false when it does not fit
+I8Plan i8_plan_rotate(const I8Plan& base, int32_t layout, int64_t n, int64_t k, int64_t batch, int sms);
+// status / wait_ns: optional device status word and bound on each pipeline wait (0 = 1 s);
+// signs: non-null to multiply by R x (the plan must come from i8_plan_rotate)
 cudaError_t launch_gemv_i8(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y, const I8Plan& pl,
-                           cudaStream_t st, uint32_t flags, uint32_t* status, uint64_t wait_ns);
+                           cudaStream_t st, uint32_t flags, uint32_t* status, uint64_t wait_ns,
+                           const int8_t* signs = nullptr);
 
 // Split-K plan of the decode GEMV for one (layout, n, k, batch) on a device with `sms` SMs.
 struct GemvPlan {
@@ -78,9 +83,10 @@ bool gemv_supported(int32_t layout, int64_t n, int64_t k, int64_t batch);
 
 // flags: TERN_GEMV_* bits of tern_gemv_ex (0 for tern_gemv).
 // status / wait_ns: optional device status word and wait bound of the kernels that wait on a pipeline.
+// signs: non-null only with an int8-plane plan from i8_plan_rotate (x is rotated in the prologue).
 cudaError_t launch_gemv(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y,
                         void* workspace, const GemvPlan& plan, cudaStream_t st, uint32_t flags = 0,
-                        uint32_t* status = nullptr, uint64_t wait_ns = 0);
+                        uint32_t* status = nullptr, uint64_t wait_ns = 0, const int8_t* signs = nullptr);
 
 // tern_gemv_noalloc's work after argument checks (scratch in a static device array).
 tern_status gemv_noalloc(const tern_matrix& W, const uint16_t* x, int batch, uint16_t* y, cudaStream_t st);

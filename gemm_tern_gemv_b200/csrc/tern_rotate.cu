@@ -11,20 +11,18 @@
 // element of a block is read before any is written, so y may alias x.
 #include <cuda_fp16.h>
 
+#include "tern_fwht.cuh"
 #include "tern_internal.cuh"
 
 namespace tern {
 namespace {
-
-constexpr int kRotBlock = 1024;
-constexpr int kRotThreads = 128;
 
 __global__ void __launch_bounds__(kRotThreads) rotate_kernel(const uint16_t* x, const int8_t* __restrict__ signs,
                                                              uint16_t* y, int64_t k, int nblk) {
   __shared__ float sh[kRotBlock];
   const int blk = blockIdx.x % nblk;
   const int64_t row = blockIdx.x / nblk;
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int t = threadIdx.x;
   const int64_t base = row * k + (int64_t)blk * kRotBlock;
   float v[8];
 #pragma unroll
@@ -33,35 +31,7 @@ __global__ void __launch_bounds__(kRotThreads) rotate_kernel(const uint16_t* x, 
     const float xv = __half2float(__ushort_as_half(x[base + i]));
     v[r] = signs[i] < 0 ? -xv : xv;
   }
-  // butterflies (a, b) -> (a + b, a - b), a the element whose index bit is clear
-#pragma unroll
-  for (int m = 1; m < 8; m <<= 1)  // index bits 7..9: register index r
-#pragma unroll
-    for (int r = 0; r < 8; r++)
-      if (!(r & m)) {
-        const float a = v[r], b = v[r | m];
-        v[r] = a + b;
-        v[r | m] = a - b;
-      }
-#pragma unroll
-  for (int m = 1; m < 32; m <<= 1)  // index bits 0..4: lane
-#pragma unroll
-    for (int r = 0; r < 8; r++) {
-      const float p = __shfl_xor_sync(0xFFFFFFFFu, v[r], m);
-      v[r] = (lane & m) ? p - v[r] : v[r] + p;
-    }
-#pragma unroll
-  for (int m = 1; m < 4; m <<= 1) {  // index bits 5..6: warp
-#pragma unroll
-    for (int r = 0; r < 8; r++) sh[t + kRotThreads * r] = v[r];
-    __syncthreads();
-#pragma unroll
-    for (int r = 0; r < 8; r++) {
-      const float p = sh[(t ^ (m << 5)) + kRotThreads * r];
-      v[r] = (warp & m) ? p - v[r] : v[r] + p;
-    }
-    __syncthreads();
-  }
+  fwht1024(v, sh, t, SyncCta{});
 #pragma unroll
   for (int r = 0; r < 8; r++)
     y[base + t + kRotThreads * r] = __half_as_ushort(__float2half_rn(v[r] * 0.03125f));

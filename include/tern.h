@@ -215,6 +215,9 @@ typedef struct tern_gemv_opts {
   uint32_t* device_status;   /* device uint32 or NULL: TERN_DEVICE_TIMEOUT is OR-ed in when a pipeline
                                 wait of the call runs out; the caller zeroes it and reads it back */
   uint64_t wait_limit_ns;    /* bound on each internal pipeline wait; 0 = the default of one second */
+  const int8_t* rotate_signs; /* device int8 [1024] or NULL: multiply by R x instead of x, R the block
+                                Hadamard rotation of tern_hadamard_rotate with these signs (k a
+                                multiple of 1024); see tern_gemv_opt */
 } tern_gemv_opts;
 
 /* tern_gemv_ex with a device status word and a wait bound. The pages ask a runtime to refuse loudly
@@ -223,10 +226,25 @@ typedef struct tern_gemv_opts {
  * (a producer that never delivers, a limit set too short) abandons its tiles, writes NaN to the
  * outputs of the rows it owns (batches 1-2), and reports TERN_DEVICE_TIMEOUT through device_status.
  * It never traps or hangs. Same arguments, result and errors as tern_gemv_ex otherwise, plus
- * TERN_ERR_ALIGNMENT for a device_status that is not 4-byte aligned. opts may be NULL (= all zero). */
+ * TERN_ERR_ALIGNMENT for a device_status that is not 4-byte aligned. opts may be NULL (= all zero).
+ *
+ * With opts->rotate_signs the call computes y = W (R x), R = H S / 32 on every 1024-element block of
+ * each row of x ("Ternary Bonsai 2 27B ..." discuss.pytorch.kr, section "블록 단위 하다마드 회전": the
+ * weights live in the rotated basis and each layer multiplies by R x; section "처리량": the sign flip
+ * and block transform precede every projection). The result equals tern_hadamard_rotate followed by
+ * tern_gemv_opt on its output. Where the int8-plane kernel runs (batches 1-2 of most shapes) it
+ * rotates x itself while it builds its activation fragments: one launch, no extra memory; elsewhere
+ * the call rotates x into the workspace first (two launches). The workspace must then hold
+ * tern_gemv_opt_workspace_bytes(W, batch, opts) bytes. Errors as above, plus TERN_ERR_INVALID_ARG
+ * for k not a multiple of 1024 with rotate_signs. */
 TERN_API tern_status tern_gemv_opt(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y,
                                    void* workspace, size_t workspace_bytes, const tern_gemv_opts* opts,
                                    void* stream);
+
+/* Workspace bytes tern_gemv_opt needs for these options (tern_gemv_workspace_bytes plus room for the
+ * rotated x when the rotation cannot be done inside the GEMV kernel); 0 on invalid arguments or when
+ * none is needed. Host only. */
+TERN_API size_t tern_gemv_opt_workspace_bytes(const tern_matrix* W, int64_t batch, const tern_gemv_opts* opts);
 
 /* Bytes of device memory tern_gemv_noalloc keeps for its split-K scratch (per GPU, for the
  * lifetime of the process). */

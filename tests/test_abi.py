@@ -259,3 +259,25 @@ def test_gemv_opt_rejects_before_launch(lib):
     assert lib.tern_gemv_opt(*args, ctypes.byref(bad_flag), None) == 1
     misaligned = T.TernGemvOptsC(0, FAKE + 2, 0)
     assert lib.tern_gemv_opt(*args, ctypes.byref(misaligned), None) == 3
+
+
+def test_rotated_gemv_checks_and_workspace(lib):
+    import gemm_tern_gemv_b200 as T
+    # K must be a multiple of the 1024-element rotation block; rejected before any CUDA call
+    m = _mat(k=1152, code_row_stride=288, scale_row_stride=16)
+    rot = T.TernGemvOptsC(0, None, 0, FAKE + 8192)
+    args = (ctypes.byref(m), ctypes.c_void_p(FAKE), 1, ctypes.c_void_p(FAKE), None, 0)
+    assert lib.tern_gemv_opt(*args, ctypes.byref(rot), None) == 1
+    assert lib.tern_gemv_opt_workspace_bytes(ctypes.byref(m), 1, ctypes.byref(rot)) == 0
+    plain = T.TernGemvOptsC(0, None, 0, None)
+    for layout, rb in ((1, 1024), (2, 832), (3, 512)):
+        for b in (1, 2, 3, 4, 17):
+            m = _mat(layout=layout, n=4096, k=4096, code_row_stride=rb, scale_row_stride=32)
+            base = lib.tern_gemv_workspace_bytes(ctypes.byref(m), b)
+            # without a rotation the size is tern_gemv_workspace_bytes'
+            assert lib.tern_gemv_opt_workspace_bytes(ctypes.byref(m), b, ctypes.byref(plain)) == base
+            need = lib.tern_gemv_opt_workspace_bytes(ctypes.byref(m), b, ctypes.byref(rot))
+            # batches 1-2 rotate inside the int8-plane kernel (binary: also 3-4, as pairs); the rest
+            # add the rotated x after the GEMV's own workspace, 256-byte aligned
+            fused = b <= 2 or (layout == 3 and b <= 4)
+            assert need == (base if fused else (base + 255) // 256 * 256 + b * 4096 * 2), (layout, b, base, need)
