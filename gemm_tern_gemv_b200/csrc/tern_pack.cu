@@ -25,6 +25,23 @@ __device__ __forceinline__ int ternary_value(uint16_t wbits, float s_abs, bool s
   return big ? (((w > 0.0f) != s_neg) ? 1 : -1) : 0;
 }
 
+// The base-3 and binary kernels decide two weights at a time, one per 16-bit lane of a 32-bit word of fp16 pairs.
+// 0xFFFF in each lane where 2|w| > |s| (s2 = |s| in both lanes): doubling an fp16 value is exact
+// unless it overflows, and then it is infinite, which is also the fp32 answer (2|w| > 65504 >= |s|);
+// NaN compares false. The caller handles s = 0 (every t is 0).
+__device__ __forceinline__ uint32_t big2(uint32_t pair, __half2 s2) {
+  __half2 a;
+  const uint32_t abs_bits = pair & 0x7FFF7FFFu;
+  a = *reinterpret_cast<const __half2*>(&abs_bits);
+  return __hgt2_mask(__hadd2(a, a), s2);
+}
+// 0xFFFF in each lane whose weight is neither +-0 nor NaN (the binary sign rule)
+__device__ __forceinline__ uint32_t nonzero2(uint32_t pair) {
+  const uint32_t abs_bits = pair & 0x7FFF7FFFu;
+  return __hgt2_mask(*reinterpret_cast<const __half2*>(&abs_bits), __float2half2_rn(0.0f));
+}
+__device__ __forceinline__ uint32_t comp(const uint4& q, int e) { return e == 0 ? q.x : e == 1 ? q.y : e == 2 ? q.z : q.w; }
+
 // ---- Q2_0_g128: chunk = 16 bytes = 64 weights, all inside one 128-weight group -------------
 __global__ void __launch_bounds__(kThreads) pack_q2_kernel(const uint16_t* __restrict__ w, int64_t w_stride,
                                                            const uint16_t* __restrict__ s, int64_t s_stride,
@@ -88,24 +105,24 @@ __global__ void __launch_bounds__(kThreads) pack_q1_kernel(const uint16_t* __res
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t row = i / chunks_per_row;
     const int ch = (int)(i - row * chunks_per_row);
-    const float sv = __half2float(__ushort_as_half(s[row * s_stride + ch]));
+    const uint16_t sb = s[row * s_stride + ch];
+    const bool s_ok = (sb & 0x7FFFu) != 0 && (sb & 0x7FFFu) <= 0x7C00u;  // s = 0 or NaN: every t is +1
+    const uint32_t sneg = (sb & 0x8000u) ? 0x80008000u : 0u;
     const uint4* src = reinterpret_cast<const uint4*>(w + row * w_stride + (int64_t)ch * kGroup);
+    uint4 v[16];
+#pragma unroll
+    for (int j = 0; j < 16; j++) v[j] = __ldg(src + j);
     uint32_t out[4];
 #pragma unroll
     for (int word = 0; word < 4; word++) {
-      uint32_t acc = 0;
+      uint32_t negs = 0;  // bit i set: weight 32 word + i has t = -1 (w * s < 0)
 #pragma unroll
-      for (int v = 0; v < 4; v++) {  // 8 weights per vector, 32 per word
-        const uint4 q = __ldg(src + 4 * word + v);
-        const uint32_t pr[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int e = 0; e < 8; e++) {
-          const float wv = __half2float(__ushort_as_half((uint16_t)(pr[e / 2] >> (16 * (e & 1)))));
-          const bool neg = (wv < 0.f && sv > 0.f) || (wv > 0.f && sv < 0.f);
-          acc |= (neg ? 0u : 1u) << (8 * v + e);
-        }
+      for (int j = 0; j < 16; j++) {  // weights 32 word + 2j (low lane) and + 1 (high lane)
+        const uint32_t pair = comp(v[4 * word + j / 4], j % 4);
+        const uint32_t x = (pair ^ sneg) & nonzero2(pair);
+        negs |= (((x >> 15) & 1u) | ((x >> 30) & 2u)) << (2 * j);
       }
-      out[word] = acc;
+      out[word] = s_ok ? ~negs : 0xFFFFFFFFu;
     }
     *reinterpret_cast<uint4*>(codes + row * c_stride + (int64_t)ch * 16) = make_uint4(out[0], out[1], out[2], out[3]);
     if (prev) {  // a weight flips when its sign bit differs from the previous packing
@@ -134,33 +151,46 @@ __global__ void __launch_bounds__(kThreads) pack_t3_kernel(const uint16_t* __res
     const int k0 = ch * 80;
     const uint16_t* wr = w + row * w_stride;
     const uint16_t* sr = s + row * s_stride;
-    uint32_t c[80];
+    // C[p]: the digits c = t + 1 of weights 2p (low lane) and 2p + 1 (high lane) of the chunk
+    uint32_t C[40];
 #pragma unroll
     for (int j = 0; j < 10; j++) {  // 10 vectors of 8 weights; K % 8 == 0 so a vector is all in or all out
       const int kv = k0 + 8 * j;
       if (kv < k) {
         const uint4 q = __ldg(reinterpret_cast<const uint4*>(wr + kv));
-        const float sv = __half2float(__ushort_as_half(sr[kv / kGroup]));  // 8 | 128: one scale per vector
-        const float s_abs = fabsf(sv);
-        const bool s_neg = sv < 0.0f;
-        const uint32_t pr[4] = {q.x, q.y, q.z, q.w};
+        const uint16_t sb = sr[kv / kGroup];  // 8 | 128: one scale per vector
+        const uint32_t sneg = (sb & 0x8000u) ? 0x80008000u : 0u;
+        const uint32_t sabs = sb & 0x7FFFu;
+        const uint32_t s2b = sabs | (sabs << 16);
+        const __half2 s2 = *reinterpret_cast<const __half2*>(&s2b);
 #pragma unroll
-        for (int e = 0; e < 8; e++)
-          c[8 * j + e] = (uint32_t)(ternary_value((e & 1) ? (uint16_t)(pr[e / 2] >> 16) : (uint16_t)(pr[e / 2] & 0xFFFFu), s_abs, s_neg) + 1);  // c = t + 1
+        for (int e = 0; e < 4; e++) {
+          const uint32_t pair = comp(q, e);
+          const uint32_t m = sabs ? big2(pair, s2) : 0u;
+          const uint32_t nb = ((pair ^ sneg) >> 15) & 0x00010001u;  // t = -1 where set (and m)
+          // c = 2 - 2 neg where |t| = 1, else 1
+          C[4 * j + e] = (m & (0x00020002u - (nb << 1))) | (~m & 0x00010001u);
+        }
       } else {
 #pragma unroll
-        for (int e = 0; e < 8; e++) c[8 * j + e] = 1u;
+        for (int e = 0; e < 4; e++) C[4 * j + e] = 0x00010001u;  // trits past K: c = 1
       }
     }
+    // byte b = sum_i c(5b + i) 3^i; a pair's lo + 3 hi is bits 16..31 of pair * 0x00010003
+    auto pair3 = [](uint32_t p) { return (p * 0x00010003u) >> 16; };
     uint32_t out[4];
 #pragma unroll
     for (int word = 0; word < 4; word++) {
       uint32_t acc = 0;
 #pragma unroll
-      for (int b = 0; b < 4; b++) {
-        const int base = 5 * (4 * word + b);
-        const uint32_t byte = c[base] + 3u * c[base + 1] + 9u * c[base + 2] + 27u * c[base + 3] + 81u * c[base + 4];
-        acc |= byte << (8 * b);
+      for (int b4 = 0; b4 < 4; b4++) {
+        const int b = 4 * word + b4, w0 = 5 * b;
+        uint32_t byte;
+        if ((w0 & 1) == 0)  // c0 c1 | c2 c3 | c4 (low lane)
+          byte = pair3(C[w0 / 2]) + 9u * pair3(C[w0 / 2 + 1]) + 81u * (C[w0 / 2 + 2] & 0xFFFFu);
+        else  // c0 (high lane) | c1 c2 | c3 c4
+          byte = (C[w0 / 2] >> 16) + 3u * pair3(C[w0 / 2 + 1]) + 27u * pair3(C[w0 / 2 + 2]);
+        acc |= byte << (8 * b4);
       }
       out[word] = acc;
     }
@@ -175,7 +205,9 @@ __global__ void __launch_bounds__(kThreads) pack_t3_kernel(const uint16_t* __res
         if (old == neu) continue;
 #pragma unroll
         for (int f = 0; f < 5; f++) {
-          flipped += (old % 3u != c[5 * b + f]) && (k0 + 5 * b + f < k);
+          const int wi = 5 * b + f;
+          const uint32_t cw = (C[wi / 2] >> (16 * (wi & 1))) & 0xFFFFu;
+          flipped += (old % 3u != cw) && (k0 + wi < k);
           old /= 3u;
         }
       }
