@@ -40,6 +40,15 @@ class TernGemvOptsC(ctypes.Structure):
                 ("rotate_signs", ctypes.c_void_p)]
 
 
+class TernGemvPlanInfoC(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_int32), ("launches", ctypes.c_int32), ("k_slices", ctypes.c_int32),
+                ("ctas_per_sm", ctypes.c_int32), ("warps", ctypes.c_int32), ("stages", ctypes.c_int32),
+                ("rotation_fused", ctypes.c_int32), ("reserved", ctypes.c_int32), ("workspace_bytes", ctypes.c_uint64)]
+
+
+GEMV_KERNELS = {1: "int8-planes", 2: "register", 3: "shared-memory", 4: "tcgen05"}
+
+
 class TernMatrixC(ctypes.Structure):
     _fields_ = [("layout", ctypes.c_int32), ("n", ctypes.c_int64), ("k", ctypes.c_int64),
                 ("codes", ctypes.c_void_p), ("code_row_stride", ctypes.c_int64),
@@ -66,6 +75,8 @@ SIGNATURES = {
                                      ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(TernGemvOptsC), ctypes.c_void_p]),
     "tern_gemv_opt_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(TernMatrixC), ctypes.c_int64,
                                                         ctypes.POINTER(TernGemvOptsC)]),
+    "tern_gemv_plan_describe": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_int64,
+                                               ctypes.POINTER(TernGemvOptsC), ctypes.POINTER(TernGemvPlanInfoC)]),
     "tern_gemv_noalloc": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                          ctypes.c_void_p]),
     "tern_gemm": (ctypes.c_int, [ctypes.POINTER(TernMatrixC), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
@@ -293,6 +304,18 @@ def gemv_opt_workspace_bytes(W: TernMatrix, batch: int, rotate_signs=None) -> in
     c = W.c()
     o = _opts(rotate_signs=rotate_signs)
     return int(lib().tern_gemv_opt_workspace_bytes(ctypes.byref(c), batch, ctypes.byref(o)))
+
+
+def gemv_plan_describe(W: TernMatrix, batch: int, rotate_signs=None, static_weights: bool = False) -> dict:
+    """tern_gemv_plan_describe: the kernel and work split tern_gemv_opt would use (host only)."""
+    c = W.c()
+    o = _opts(static_weights, None, 0, rotate_signs)
+    info = TernGemvPlanInfoC()
+    _check(lib().tern_gemv_plan_describe(ctypes.byref(c), batch, ctypes.byref(o), ctypes.byref(info)),
+           "tern_gemv_plan_describe")
+    d = {f: getattr(info, f) for f, _ in TernGemvPlanInfoC._fields_ if f != "reserved"}
+    d["kernel"] = GEMV_KERNELS.get(d["kernel"], d["kernel"])
+    return d
 
 
 def gemv_opt(W: TernMatrix, x, y=None, workspace=None, static_weights: bool = False, status=None,

@@ -211,6 +211,49 @@ tern_status tern_gemv_opt(const tern_matrix* W, const uint16_t* x, int64_t batch
   return from_cuda(launch_gemv(*W, x, (int)batch, y, workspace, op.plan, st, flags, status, wait_ns, signs));
 }
 
+tern_status tern_gemv_plan_describe(const tern_matrix* W, int64_t batch, const tern_gemv_opts* opts,
+                                    tern_gemv_plan_info* out) {
+  if (!out) return TERN_ERR_INVALID_ARG;
+  const uint32_t flags = opts ? opts->flags : 0u;
+  const int8_t* signs = opts ? opts->rotate_signs : nullptr;
+  if (flags & ~(uint32_t)TERN_GEMV_STATIC_WEIGHTS) return TERN_ERR_INVALID_ARG;
+  tern_status s = check_matrix(W);
+  if (s != TERN_OK) return s;
+  if (batch < 1 || batch > TERN_GEMV_MAX_BATCH) return TERN_ERR_INVALID_ARG;
+  if (signs && W->k % kRotBlock) return TERN_ERR_INVALID_ARG;
+  if (!gemv_supported(W->layout, W->n, W->k, batch)) return TERN_ERR_UNSUPPORTED;
+  const OptPlan op = opt_plan(*W, batch, signs != nullptr);
+  const GemvPlan& p = op.plan;
+  tern_gemv_plan_info info{};
+  if (p.i8) {
+    info.kernel = TERN_GEMV_KERNEL_INT8_PLANES;
+    info.launches = (int32_t)((batch + 1) / 2);  // one launch per pair of rows
+    info.k_slices = p.i8p.ks;
+    info.ctas_per_sm = p.i8p.cps;
+    info.warps = p.i8p.nw;
+    info.stages = p.i8p.stages;
+  } else if (p.gemm) {
+    info.kernel = TERN_GEMV_KERNEL_TCGEN05;
+    info.launches = 1;
+    info.k_slices = 1;
+  } else if (p.reg) {
+    info.kernel = TERN_GEMV_KERNEL_REGISTER;
+    info.launches = W->layout == TERN_Q1_0_G128 ? (int32_t)((batch + kBinChunk - 1) / kBinChunk) : 1;
+    info.k_slices = p.splits;
+    info.ctas_per_sm = p.warps == 8 ? 2 : 1;
+    info.warps = p.warps;
+  } else {
+    info.kernel = TERN_GEMV_KERNEL_SHARED;
+    info.launches = 1;
+    info.k_slices = p.splits;
+  }
+  info.rotation_fused = op.fused ? 1 : 0;
+  if (signs && !op.fused) info.launches += 1;  // tern_hadamard_rotate's kernel into the workspace
+  info.workspace_bytes = op.ws;
+  *out = info;
+  return TERN_OK;
+}
+
 tern_status tern_gemv_noalloc(const tern_matrix* W, const uint16_t* x, int64_t batch, uint16_t* y, void* stream) {
   tern_status s = check_matrix(W);
   if (s != TERN_OK) return s;

@@ -1263,7 +1263,6 @@ cudaError_t launch_reg(const CUtensorMap& tc, const CUtensorMap& ts, const Args&
 #define TERN_REG_STAGES_T3 3
 #endif
 constexpr int kRegRT = TERN_REG_RT;
-constexpr int kBinChunk = 2;  // batch rows per launch of the binary register kernel
 constexpr int kRegStagesQ2 = TERN_REG_STAGES_Q2;
 constexpr int kRegStagesT3 = TERN_REG_STAGES_T3;
 

@@ -13,6 +13,7 @@
 namespace tern {
 
 constexpr int kGroup = TERN_GROUP;
+constexpr int kBinChunk = 2;  // batch rows per launch of the binary register kernel
 
 // Minimum packed row stride in bytes (see tern_row_bytes); -1 on invalid arguments.
 int64_t row_bytes(int32_t layout, int64_t k);

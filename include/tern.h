@@ -338,6 +338,30 @@ TERN_API tern_status tern_hadamard_rotate(const uint16_t* x, int64_t batch, int6
  * invalid_count > 0, else TERN_OK. Host only; makes no CUDA call. */
 TERN_API tern_status tern_device_result(uint32_t device_status, int64_t invalid_count);
 
+/* What a tern_gemv_opt call with these arguments would launch: the kernel, its work split and the
+ * workspace it needs. Host only (no CUDA call beyond reading the device's SM count once); for tests,
+ * logs and tuning. This entry point is an engineering addition; the pages have no counterpart to it. */
+typedef struct tern_gemv_plan_info {
+  int32_t kernel;          /* TERN_GEMV_KERNEL_*: the kernel that computes the product */
+  int32_t launches;        /* kernel launches of the call, a rotation into the workspace included */
+  int32_t k_slices;        /* K split: CTAs of a cluster (int8-plane kernel) or slices (others); 1 = none */
+  int32_t ctas_per_sm;     /* CTAs per SM (int8-plane and register kernels; 0 = not fixed) */
+  int32_t warps;           /* consumer warps per CTA (int8-plane and register kernels; else 0) */
+  int32_t stages;          /* TMA ring stages (int8-plane kernel; else 0) */
+  int32_t rotation_fused;  /* 1: opts->rotate_signs is applied inside the GEMV kernel's prologue */
+  int32_t reserved;
+  uint64_t workspace_bytes; /* = tern_gemv_opt_workspace_bytes */
+} tern_gemv_plan_info;
+#define TERN_GEMV_KERNEL_INT8_PLANES 1  /* batch 1-2: int8 mma.sync on TMA-streamed tiles */
+#define TERN_GEMV_KERNEL_REGISTER 2     /* fp16 mma.sync, decode in registers from TMA windows */
+#define TERN_GEMV_KERNEL_SHARED 3       /* fp16 mma.sync, decode through shared memory */
+#define TERN_GEMV_KERNEL_TCGEN05 4      /* the tcgen05 GEMM kernel (batches >= 17, N % 8 == 0) */
+
+/* Fills *out for tern_gemv_opt(W, x, batch, y, ..., opts, ...). Errors: those of tern_gemv_opt's
+ * argument checks on W, batch and opts (x, y and the workspace are not looked at); out != NULL. */
+TERN_API tern_status tern_gemv_plan_describe(const tern_matrix* W, int64_t batch, const tern_gemv_opts* opts,
+                                             tern_gemv_plan_info* out);
+
 /* Static description of a status code (never NULL). */
 TERN_API const char* tern_status_string(tern_status status);
 

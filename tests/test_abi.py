@@ -281,3 +281,64 @@ def test_rotated_gemv_checks_and_workspace(lib):
             # add the rotated x after the GEMV's own workspace, 256-byte aligned
             fused = b <= 2 or (layout == 3 and b <= 4)
             assert need == (base if fused else (base + 255) // 256 * 256 + b * 4096 * 2), (layout, b, base, need)
+
+
+def _describe(lib, layout, n, k, b, signs=None):
+    import gemm_tern_gemv_b200 as T
+    rb = {1: k // 4, 2: -(-(-(-k // 5)) // 16) * 16, 3: k // 8}[layout]
+    m = _mat(layout=layout, n=n, k=k, code_row_stride=rb, scale_row_stride=max(8, -(-(k // 128) // 8) * 8))
+    o = T.TernGemvOptsC(0, None, 0, signs)
+    info = T.TernGemvPlanInfoC()
+    st = lib.tern_gemv_plan_describe(ctypes.byref(m), b, ctypes.byref(o), ctypes.byref(info))
+    return st, info, m, o
+
+
+def test_plan_description_follows_the_planner_rules(lib):
+    # (148-SM B200 planning without a GPU) the int8-plane kernel takes batches 1-2 with one K slice
+    # when it fits: two CTAs of 8 warps per SM from 14 row tiles per SM, 8 warps for at most two tiles,
+    # else one CTA of 16; a slice that does not fit splits K over a pair of CTAs with 12 warps
+    expect = {  # (layout, n, k, batch): (k_slices, ctas_per_sm, warps)
+        (1, 4096, 4096, 1): (1, 1, 8), (1, 24576, 4096, 1): (1, 1, 16), (2, 24576, 4096, 1): (1, 1, 16),
+        (2, 151936, 4096, 1): (1, 2, 8), (1, 34816, 5120, 1): (1, 2, 8), (2, 4096, 12288, 1): (2, 1, 12),
+        (1, 5120, 17408, 1): (2, 1, 12), (2, 5120, 17408, 1): (2, 1, 12), (3, 24576, 4096, 1): (1, 1, 16),
+    }
+    for (layout, n, k, b), (ks, cps, nw) in expect.items():
+        st, info, m, _ = _describe(lib, layout, n, k, b)
+        assert st == 0
+        assert info.kernel == 1 and info.launches == 1, (layout, n, k, b)
+        assert (info.k_slices, info.ctas_per_sm, info.warps) == (ks, cps, nw), (layout, n, k, b, info.k_slices,
+                                                                                info.ctas_per_sm, info.warps)
+        assert info.stages >= 2 and info.workspace_bytes == lib.tern_gemv_workspace_bytes(ctypes.byref(m), b) == 0
+    # batch 2 of the LM head stays on the older kernels (a K split there would keep a partial per tile)
+    st, info, _, _ = _describe(lib, 2, 151936, 4096, 2)
+    assert st == 0 and info.kernel != 1
+    # binary batches 3-4 run as pairs of rows on the int8-plane kernel; batch 17 with N % 8 == 0 on tcgen05
+    st, info, _, _ = _describe(lib, 3, 4096, 4096, 3)
+    assert st == 0 and info.kernel == 1 and info.launches == 2
+    for layout in (1, 2, 3):
+        st, info, _, _ = _describe(lib, layout, 4096, 4096, 17)
+        assert st == 0 and info.kernel == 4 and info.launches == 1
+    # every described plan is self-consistent over a sweep of shapes and batches
+    for layout in (1, 2, 3):
+        for n in (1, 17, 4096, 34816):
+            for k in (1024, 4096, 5120, 17408):
+                for b in (1, 2, 3, 8, 16, 64):
+                    st, info, m, o = _describe(lib, layout, n, k, b)
+                    assert st == 0
+                    assert 1 <= info.kernel <= 4 and info.launches >= 1 and info.k_slices >= 1
+                    assert info.workspace_bytes == lib.tern_gemv_opt_workspace_bytes(ctypes.byref(m), b, ctypes.byref(o))
+                    if info.kernel == 1:
+                        assert b <= 2 or layout == 3
+                        assert info.k_slices in (1, 2, 4) and info.ctas_per_sm in (1, 2) and info.stages >= 2
+                        assert info.warps <= (8 if info.ctas_per_sm == 2 else 17)
+
+
+def test_plan_description_of_the_rotation(lib):
+    signs = FAKE + 8192
+    st, info, m, o = _describe(lib, 1, 4096, 4096, 1, signs)
+    assert st == 0 and info.rotation_fused == 1 and info.launches == 1 and info.workspace_bytes == 0
+    st, info, m, o = _describe(lib, 1, 4096, 4096, 3, signs)  # register kernel: rotate into the workspace
+    assert st == 0 and info.rotation_fused == 0 and info.launches == 2
+    assert info.workspace_bytes == lib.tern_gemv_opt_workspace_bytes(ctypes.byref(m), 3, ctypes.byref(o)) > 0
+    st, info, _, _ = _describe(lib, 1, 4096, 1152, 1, signs)
+    assert st == 1  # K is not a multiple of the 1024-element rotation block
