@@ -179,7 +179,8 @@ TERN_API size_t tern_gemv_workspace_bytes(const tern_matrix* W, int64_t batch);
  * packed codes are read directly and unpack and group scale are fused, section "하이브리드 어텐션을
  * 위한 저비트 커널"); the activations' own precision is kept (x exact as int8 planes or fp16), fp32
  * accumulation, fp16 result. Batches 1-2 run on int8 mma.sync kernels fed by TMA (K split over a
- * cluster for narrow matrices); batches 3-16 on fp16 mma.sync kernels; batches of 17 or more with
+ * cluster for narrow matrices; rows that are not whole 64-byte (Q2) / 32-byte units, and batch-2 K
+ * splits of tall matrices, use the fp16 kernels); batches 3-16 on fp16 mma.sync kernels; batches of 17 or more with
  * n % 8 == 0 on the tcgen05 kernel of tern_gemm (no workspace), as do Q1_0_g128 batches of 5 or
  * more with n % 8 == 0. Other Q1_0_g128 batches run as one launch per two rows of x.
  * The result of a call depends only on (W, x, batch) and the device.
@@ -196,11 +197,12 @@ TERN_API tern_status tern_gemv(const tern_matrix* W, const uint16_t* x, int64_t 
                       void* workspace, size_t workspace_bytes, void* stream);
 
 /* Flag of tern_gemv_ex: nothing that may still be running on the GPU when the call is made writes
- * W's codes or scales (the usual case in a decode loop over fixed weights). The register-decode GEMV
- * (batches 1-4 of Q2_0_g128, 1-2 of base-3, those of Q1_0_g128 not taken by the GEMM) is then launched as a
- * programmatic dependent of the preceding kernel on the stream: its CTAs may start as the preceding
- * grid's CTAs leave their SMs and begin streaming W, while x, y and the workspace are still only
- * touched after the preceding grid has completed. Other paths ignore the flag. */
+ * W's codes or scales (the usual case in a decode loop over fixed weights). The int8-plane GEMV
+ * (batches 1-2, and Q1_0_g128 pairs of rows) and the register-decode GEMV (batches 3-4 of Q2_0_g128
+ * and the shapes the int8-plane kernel does not take) are launched as programmatic dependents of the
+ * preceding kernel on the stream; with this flag their CTAs request W's first tiles as soon as they
+ * start, while the preceding grid finishes, and x, y and the workspace are still only touched after
+ * the preceding grid has completed. Other paths ignore the flag. */
 #define TERN_GEMV_STATIC_WEIGHTS 1u
 
 /* tern_gemv with flags (0 or TERN_GEMV_STATIC_WEIGHTS); same arguments, result and errors, plus
