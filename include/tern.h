@@ -197,12 +197,12 @@ TERN_API tern_status tern_gemv(const tern_matrix* W, const uint16_t* x, int64_t 
                       void* workspace, size_t workspace_bytes, void* stream);
 
 /* Flag of tern_gemv_ex: nothing that may still be running on the GPU when the call is made writes
- * W's codes or scales (the usual case in a decode loop over fixed weights). The int8-plane GEMV
- * (batches 1-2, and Q1_0_g128 pairs of rows) and the register-decode GEMV (batches 3-4 of Q2_0_g128
- * and the shapes the int8-plane kernel does not take) are launched as programmatic dependents of the
- * preceding kernel on the stream; with this flag their CTAs request W's first tiles as soon as they
- * start, while the preceding grid finishes, and x, y and the workspace are still only touched after
- * the preceding grid has completed. Other paths ignore the flag. */
+ * W's codes or scales (the usual case in a decode loop over fixed weights). With it, the int8-plane
+ * GEMV (batches 1-2, and Q1_0_g128 pairs of rows; always launched as a programmatic dependent of the
+ * preceding kernel on the stream) and the register-decode GEMV (batches 3-4 of Q2_0_g128 and the
+ * shapes the int8-plane kernel does not take; then launched as one) request W's first tiles as soon
+ * as their CTAs start, while the preceding grid finishes; x, y and the workspace are only touched
+ * after the preceding grid has completed. Other paths ignore the flag. */
 #define TERN_GEMV_STATIC_WEIGHTS 1u
 
 /* tern_gemv with flags (0 or TERN_GEMV_STATIC_WEIGHTS); same arguments, result and errors, plus
